@@ -1,0 +1,359 @@
+/*
+ * CPU oracle for the fused MoE expert-FFN forward.
+ *
+ * TEST INFRASTRUCTURE.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference legs of bench.py load this library.  The product
+ * path (the CUDA library and its Python binding) never does.
+ *
+ * Plain C, double accumulation, loops written in the order of the definitions
+ * on the pages; no blocking, no fusion, no reordering.  Sources:
+ *   [RFC] "[RFC] Fused W8A8 MoE megakernel on H20": Background (the five local
+ *         steps: count/gather, gate/up GroupGEMM, SiLU x gate + requant, down
+ *         GroupGEMM, top-k weighted reduction) and Design (histogram, prefix
+ *         sums, row-to-token mapping).
+ *   [PFM] "Prime Flash MoE: Fused MoE Kernels for Blackwell": intro (SwiGLU
+ *         consumed from the accumulator, mxfp8 requant of the intermediate),
+ *         API (moe_align outputs), Shapes (x, w1, w2, out, topk_weights, the
+ *         flattened token*top_k+route ids padded with -1), Scale layout
+ *         (mxfp8) (row-major activation scales, 512-byte blocked weight-scale
+ *         tiles of 128 MN x 128 K, OCP MX quantiser).
+ * Readings where the pages are silent (gate = rows [0, N/2) of w1, stable
+ * order inside an expert segment, -1 in unused capacity, e8m0 byte 0 for an
+ * all-zero block, saturation to +-448, round-to-nearest-even everywhere) are
+ * listed in the design notes and repeated beside the code that takes them.
+ *
+ * Parity status: every function here is pinned by tests/test_oracle_*.py
+ * (closed forms, invariants, brute force, torch float64 / float8 library
+ * routines on special cases).  Nothing is "parity unpinned".
+ */
+#include "oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ====================================================================== */
+/* scalar formats                                                          */
+/* ====================================================================== */
+
+double orc_bf16_to_double(uint16_t bits) {
+  uint32_t u = (uint32_t)bits << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* Round a double to the nearest bfloat16 (8 significant bits, fp32 exponent
+ * range), ties to even, overflow to infinity (IEEE default rounding). */
+uint16_t orc_double_to_bf16(double x) {
+  if (isnan(x)) return 0x7FC0;
+  if (x == 0.0) return signbit(x) ? 0x8000 : 0x0000;
+  int e;
+  (void)frexp(x, &e);               /* |x| = m * 2^e, 0.5 <= m < 1 */
+  int qe = e < -125 ? -125 : e;     /* smallest normal binade is 2^-126 */
+  double quantum = ldexp(1.0, qe - 8);
+  double q = nearbyint(x / quantum) * quantum;   /* default mode: ties-to-even */
+  const double maxv = ldexp(255.0, 127 - 7);     /* (2 - 2^-7) * 2^127 */
+  float f;
+  if (fabs(q) > maxv) f = (float)(q > 0 ? INFINITY : -INFINITY);
+  else f = (float)q;                              /* exact: q has <= 8 bits */
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  return (uint16_t)(u >> 16);
+}
+
+/* OCP E4M3 ("fn" flavour): bias 7, 3 mantissa bits, no infinities,
+ * S.1111.111 is NaN, largest finite 448, subnormals m * 2^-9. */
+double orc_e4m3_to_double(uint8_t code) {
+  int s = code >> 7, ex = (code >> 3) & 0xF, m = code & 7;
+  if (ex == 0xF && m == 7) return NAN;
+  double v = ex == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, ex - 7);
+  return s ? -v : v;
+}
+
+/* Round to nearest e4m3, ties to even, magnitudes beyond 448 saturate. */
+uint8_t orc_double_to_e4m3(double x) {
+  if (isnan(x)) return 0x7F;
+  uint8_t sign = signbit(x) ? 0x80 : 0x00;
+  double a = fabs(x);
+  if (a == 0.0) return sign;
+  int e;
+  (void)frexp(a, &e);               /* 2^(e-1) <= a < 2^e */
+  int qe = e < -5 ? -5 : e;         /* smallest normal binade 2^-6 */
+  double quantum = ldexp(1.0, qe - 4);            /* 4 significant bits */
+  double q = nearbyint(a / quantum) * quantum;
+  if (q > 448.0) q = 448.0;
+  /* encode the (exactly representable) magnitude q */
+  if (q < ldexp(1.0, -6)) {                       /* subnormal or zero */
+    int m = (int)nearbyint(q / ldexp(1.0, -9));
+    return sign | (uint8_t)m;
+  }
+  int qe2;
+  double mq = frexp(q, &qe2);                     /* q = mq * 2^qe2 */
+  int ex = qe2 - 1 + 7;                            /* biased exponent */
+  int m = (int)nearbyint((mq * 2.0 - 1.0) * 8.0);
+  return sign | (uint8_t)(ex << 3) | (uint8_t)m;
+}
+
+double orc_e8m0_to_double(uint8_t code) {
+  if (code == 0xFF) return NAN;
+  return ldexp(1.0, (int)code - 127);
+}
+
+/* OCP MX v1.0 shared scale: X = 2^(floor(log2(amax)) - emax_elem), with
+ * emax_elem = 8 for E4M3, stored as the biased e8m0 byte.  An all-zero block
+ * takes byte 0 (reading: the spec leaves log2(0) open).  Clamped to the
+ * finite e8m0 range [2^-127, 2^127]. */
+uint8_t orc_mx_scale_byte(float amax) {
+  if (!(amax > 0.0f)) return 0;
+  int e;
+  (void)frexp((double)amax, &e);    /* floor(log2(amax)) = e - 1, exact */
+  int shared = (e - 1) - 8;
+  if (shared < -127) shared = -127;
+  if (shared > 127) shared = 127;
+  return (uint8_t)(shared + 127);
+}
+
+void orc_mx_quantize(const float* v, int64_t n, uint8_t* codes, uint8_t* scales) {
+  for (int64_t b = 0; b < n / 32; ++b) {
+    float amax = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+      float a = fabsf(v[b * 32 + i]);
+      if (a > amax) amax = a;
+    }
+    uint8_t sb = orc_mx_scale_byte(amax);
+    scales[b] = sb;
+    double X = orc_e8m0_to_double(sb);
+    for (int i = 0; i < 32; ++i) codes[b * 32 + i] = orc_double_to_e4m3((double)v[b * 32 + i] / X);
+  }
+}
+
+/* ====================================================================== */
+/* planner: moe_align                                                     */
+/* [RFC] Design: expert histogram, prefix sums, row-to-token mapping.     */
+/* [PFM] API / Shapes: sorted_token_ids holds flattened token*top_k+route */
+/* ids grouped by expert and padded to block_m with -1; expert_ids gives  */
+/* the expert of each block_m block; num_tokens_post_padded the total.    */
+/* ====================================================================== */
+
+int64_t orc_align_capacity(int T, int top_k, int E, int block_m) {
+  return (int64_t)T * top_k + (int64_t)E * (block_m - 1);
+}
+
+int orc_moe_align(const int32_t* topk_ids, int T, int top_k, int E, int block_m,
+                  int32_t* sorted_token_ids, int32_t* expert_ids,
+                  int32_t* num_tokens_post_padded, int64_t capacity) {
+  const int64_t R = (int64_t)T * top_k;
+  int64_t* count = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+  int64_t* off = (int64_t*)calloc((size_t)E + 1, sizeof(int64_t));
+  int64_t* cursor = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+  if (!count || !off || !cursor) { free(count); free(off); free(cursor); return -1; }
+
+  /* step 1: histogram (ids outside [0, E) are not routed anywhere) */
+  for (int64_t i = 0; i < R; ++i) {
+    int e = topk_ids[i];
+    if (e >= 0 && e < E) count[e] += 1;
+  }
+  /* step 2: exclusive prefix sum of counts padded up to block_m */
+  off[0] = 0;
+  for (int e = 0; e < E; ++e) {
+    int64_t padded = (count[e] + block_m - 1) / block_m * block_m;
+    off[e + 1] = off[e] + padded;
+  }
+  const int64_t ntpp = off[E];
+  if (ntpp > capacity) { free(count); free(off); free(cursor); return -2; }
+  *num_tokens_post_padded = (int32_t)ntpp;
+
+  /* step 3: row-to-token map.  Every slot starts as -1 (padding and unused
+   * capacity); ids are placed in ascending flattened order, so each expert
+   * segment is stable (reading: the pages fix no order inside a segment). */
+  for (int64_t p = 0; p < capacity; ++p) sorted_token_ids[p] = -1;
+  for (int64_t i = 0; i < R; ++i) {
+    int e = topk_ids[i];
+    if (e < 0 || e >= E) continue;
+    sorted_token_ids[off[e] + cursor[e]] = (int32_t)i;
+    cursor[e] += 1;
+  }
+  /* expert of every block; -1 for blocks past the last padded segment */
+  const int64_t nblk_cap = (capacity + block_m - 1) / block_m;
+  for (int64_t b = 0; b < nblk_cap; ++b) expert_ids[b] = -1;
+  for (int e = 0; e < E; ++e)
+    for (int64_t p = off[e]; p < off[e + 1]; p += block_m) expert_ids[p / block_m] = e;
+
+  free(count); free(off); free(cursor);
+  return 0;
+}
+
+/* ====================================================================== */
+/* [PFM] Scale layout (mxfp8): weight scales reordered into a sequence of */
+/* 512-byte tiles, each covering 128 MN x 128 K (= 4 scale bytes along K). */
+/* Tile order: expert, then MN tile, then K tile.  Inside a tile row r and */
+/* scale column c sit at byte (r % 32) * 16 + (r / 32) * 4 + c (reading:  */
+/* the layout the Blackwell block-scaled MMA consumes).  Pad bytes are 0. */
+/* ====================================================================== */
+
+int64_t orc_pack_scales_bytes(int E, int MN, int KS) {
+  int64_t MT = (MN + 127) / 128, KT = (KS + 3) / 4;
+  return (int64_t)E * MT * KT * 512;
+}
+
+static int64_t blocked_offset(int e, int row, int col, int MN, int KS) {
+  int64_t MT = (MN + 127) / 128, KT = (KS + 3) / 4;
+  int mt = row / 128, r = row % 128, kt = col / 4, c = col % 4;
+  return (((int64_t)e * MT + mt) * KT + kt) * 512 + (r % 32) * 16 + (r / 32) * 4 + c;
+}
+
+void orc_pack_scales_blocked(const uint8_t* in, uint8_t* out, int E, int MN, int KS) {
+  memset(out, 0, (size_t)orc_pack_scales_bytes(E, MN, KS));
+  for (int e = 0; e < E; ++e)
+    for (int row = 0; row < MN; ++row)
+      for (int col = 0; col < KS; ++col)
+        out[blocked_offset(e, row, col, MN, KS)] = in[((int64_t)e * MN + row) * KS + col];
+}
+
+void orc_unpack_scales_blocked(const uint8_t* in, uint8_t* out, int E, int MN, int KS) {
+  for (int e = 0; e < E; ++e)
+    for (int row = 0; row < MN; ++row)
+      for (int col = 0; col < KS; ++col)
+        out[((int64_t)e * MN + row) * KS + col] = in[blocked_offset(e, row, col, MN, KS)];
+}
+
+/* ====================================================================== */
+/* expert FFN                                                             */
+/* ====================================================================== */
+
+static double silu(double g) { return g / (1.0 + exp(-g)); }
+
+static void set_threads(int nthreads) {
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+  (void)nthreads;
+#endif
+}
+
+int orc_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+/* bf16 path ([PFM] intro and Shapes; [RFC] Background steps 2-5), one token
+ * at a time, straight from the definition:
+ *   for each route j of token t, e = topk_ids[t, j]:
+ *     H = w1[e] x[t]                      (N values; gate = H[0:I], up = H[I:N])
+ *     a_i = bf16( silu(H_i) * H_{I+i} )   (activations are bf16 on this path)
+ *     Y = w2[e] a                         (K values)
+ *     acc += topk_weights[t, j] * Y
+ *   out[t] = bf16(acc)                                                      */
+void orc_fused_moe_bf16(const uint16_t* x, const uint16_t* w1, const uint16_t* w2,
+                        const int32_t* topk_ids, const float* topk_weights,
+                        int T, int K, int N, int E, int top_k,
+                        const int32_t* tokens, int n_tokens, uint16_t* out, int nthreads) {
+  const int I = N / 2;
+  const int count = tokens ? n_tokens : T;
+  set_threads(nthreads);
+#pragma omp parallel
+  {
+    double* H = (double*)malloc(sizeof(double) * (size_t)N);
+    double* a = (double*)malloc(sizeof(double) * (size_t)I);
+    double* acc = (double*)malloc(sizeof(double) * (size_t)K);
+#pragma omp for schedule(dynamic, 1)
+    for (int idx = 0; idx < count; ++idx) {
+      const int t = tokens ? tokens[idx] : idx;
+      for (int h = 0; h < K; ++h) acc[h] = 0.0;
+      for (int j = 0; j < top_k; ++j) {
+        const int e = topk_ids[(int64_t)t * top_k + j];
+        if (e < 0 || e >= E) continue;
+        const uint16_t* W1 = w1 + (int64_t)e * N * K;
+        const uint16_t* W2 = w2 + (int64_t)e * K * I;
+        for (int n = 0; n < N; ++n) {
+          double s = 0.0;
+          for (int k = 0; k < K; ++k)
+            s += orc_bf16_to_double(W1[(int64_t)n * K + k]) * orc_bf16_to_double(x[(int64_t)t * K + k]);
+          H[n] = s;
+        }
+        for (int i = 0; i < I; ++i)
+          a[i] = orc_bf16_to_double(orc_double_to_bf16(silu(H[i]) * H[I + i]));
+        const double wgt = (double)topk_weights[(int64_t)t * top_k + j];
+        for (int h = 0; h < K; ++h) {
+          double s = 0.0;
+          for (int i = 0; i < I; ++i) s += orc_bf16_to_double(W2[(int64_t)h * I + i]) * a[i];
+          acc[h] += wgt * s;
+        }
+      }
+      for (int h = 0; h < K; ++h) out[(int64_t)t * K + h] = orc_double_to_bf16(acc[h]);
+    }
+    free(H); free(a); free(acc);
+  }
+}
+
+/* mxfp8 path ([PFM] intro: e4m3 values with e8m0 block scales on both
+ * operands, intermediate requantised to mxfp8 before the down projection;
+ * Scale layout (mxfp8): block size 32 along K).  Operands are dequantised
+ * exactly (code value * 2^(scale-127)).  The SwiGLU value is rounded to
+ * fp32 (the precision the kernel holds it in), then requantised per row in
+ * blocks of 32 along the intermediate dimension with the OCP MX rule, and the
+ * down projection uses the dequantised requantised values.                 */
+void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
+                         const uint8_t* w1, const uint8_t* w1_scales,
+                         const uint8_t* w2, const uint8_t* w2_scales,
+                         const int32_t* topk_ids, const float* topk_weights,
+                         int T, int K, int N, int E, int top_k,
+                         const int32_t* tokens, int n_tokens, uint16_t* out, int nthreads) {
+  const int I = N / 2;
+  const int KS = K / 32, IS = I / 32;
+  const int count = tokens ? n_tokens : T;
+  set_threads(nthreads);
+#pragma omp parallel
+  {
+    double* xd = (double*)malloc(sizeof(double) * (size_t)K);
+    double* H = (double*)malloc(sizeof(double) * (size_t)N);
+    float* af = (float*)malloc(sizeof(float) * (size_t)I);
+    uint8_t* aq = (uint8_t*)malloc((size_t)I);
+    uint8_t* as = (uint8_t*)malloc((size_t)IS);
+    double* a = (double*)malloc(sizeof(double) * (size_t)I);
+    double* acc = (double*)malloc(sizeof(double) * (size_t)K);
+#pragma omp for schedule(dynamic, 1)
+    for (int idx = 0; idx < count; ++idx) {
+      const int t = tokens ? tokens[idx] : idx;
+      for (int k = 0; k < K; ++k)
+        xd[k] = orc_e4m3_to_double(x[(int64_t)t * K + k]) *
+                orc_e8m0_to_double(x_scales[(int64_t)t * KS + k / 32]);
+      for (int h = 0; h < K; ++h) acc[h] = 0.0;
+      for (int j = 0; j < top_k; ++j) {
+        const int e = topk_ids[(int64_t)t * top_k + j];
+        if (e < 0 || e >= E) continue;
+        const uint8_t* W1 = w1 + (int64_t)e * N * K;
+        const uint8_t* S1 = w1_scales + (int64_t)e * N * KS;
+        const uint8_t* W2 = w2 + (int64_t)e * K * I;
+        const uint8_t* S2 = w2_scales + (int64_t)e * K * IS;
+        for (int n = 0; n < N; ++n) {
+          double s = 0.0;
+          for (int k = 0; k < K; ++k)
+            s += orc_e4m3_to_double(W1[(int64_t)n * K + k]) *
+                 orc_e8m0_to_double(S1[(int64_t)n * KS + k / 32]) * xd[k];
+          H[n] = s;
+        }
+        for (int i = 0; i < I; ++i) af[i] = (float)(silu(H[i]) * H[I + i]);
+        orc_mx_quantize(af, I, aq, as);
+        for (int i = 0; i < I; ++i) a[i] = orc_e4m3_to_double(aq[i]) * orc_e8m0_to_double(as[i / 32]);
+        const double wgt = (double)topk_weights[(int64_t)t * top_k + j];
+        for (int h = 0; h < K; ++h) {
+          double s = 0.0;
+          for (int i = 0; i < I; ++i)
+            s += orc_e4m3_to_double(W2[(int64_t)h * I + i]) *
+                 orc_e8m0_to_double(S2[(int64_t)h * IS + i / 32]) * a[i];
+          acc[h] += wgt * s;
+        }
+      }
+      for (int h = 0; h < K; ++h) out[(int64_t)t * K + h] = orc_double_to_bf16(acc[h]);
+    }
+    free(xd); free(H); free(af); free(aq); free(as); free(a); free(acc);
+  }
+}
