@@ -71,9 +71,9 @@ def _load():
         lib.orc_pack_scales_blocked.restype = None
         lib.orc_unpack_scales_blocked.argtypes = [P, P, I, I, I]
         lib.orc_unpack_scales_blocked.restype = None
-        lib.orc_fused_moe_bf16.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, I]
+        lib.orc_fused_moe_bf16.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, P, I]
         lib.orc_fused_moe_bf16.restype = None
-        lib.orc_fused_moe_mxfp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, I, P, I]
+        lib.orc_fused_moe_mxfp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, I, P, P, I]
         lib.orc_fused_moe_mxfp8.restype = None
         lib.orc_max_threads.argtypes = []
         lib.orc_max_threads.restype = I
@@ -166,10 +166,12 @@ def _tokens_arg(tokens, T):
     return t, int(t.size)
 
 
-def fused_moe_bf16(x, w1, w2, topk_ids, topk_weights, tokens=None, nthreads: int = 0):
+def fused_moe_bf16(x, w1, w2, topk_ids, topk_weights, tokens=None, nthreads: int = 0, unrounded: bool = False):
     """x (T,K) uint16 bf16 bits, w1 (E,N,K), w2 (E,K,N/2) -> out (T,K) uint16 bits.
 
-    Rows of tokens not listed in ``tokens`` are left zero."""
+    Rows of tokens not listed in ``tokens`` are left zero.  With
+    ``unrounded=True`` also returns out before its final bf16 rounding
+    (float64, (T, K))."""
     x = np.ascontiguousarray(x, dtype=np.uint16)
     w1 = np.ascontiguousarray(w1, dtype=np.uint16)
     w2 = np.ascontiguousarray(w2, dtype=np.uint16)
@@ -181,14 +183,18 @@ def fused_moe_bf16(x, w1, w2, topk_ids, topk_weights, tokens=None, nthreads: int
     top_k = ids.shape[1]
     t, n = _tokens_arg(tokens, T)
     out = np.zeros((T, K), dtype=np.uint16)
+    f64 = np.zeros((T, K), dtype=np.float64) if unrounded else None
     _load().orc_fused_moe_bf16(_ptr(x), _ptr(w1), _ptr(w2), _ptr(ids), _ptr(tw), T, K, N, E, top_k,
-                               None if t is None else _ptr(t), n, _ptr(out), int(nthreads))
-    return out
+                               None if t is None else _ptr(t), n, _ptr(out),
+                               None if f64 is None else _ptr(f64), int(nthreads))
+    return (out, f64) if unrounded else out
 
 
 def fused_moe_mxfp8(x, x_scales, w1, w1_scales, w2, w2_scales, topk_ids, topk_weights,
-                    tokens=None, nthreads: int = 0):
-    """All scales ROW-MAJOR: x_scales (T,K/32), w1_scales (E,N,K/32), w2_scales (E,K,N/64)."""
+                    tokens=None, nthreads: int = 0, unrounded: bool = False):
+    """All scales ROW-MAJOR: x_scales (T,K/32), w1_scales (E,N,K/32), w2_scales (E,K,N/64).
+
+    With ``unrounded=True`` also returns out before its final bf16 rounding."""
     arrs = [np.ascontiguousarray(a, dtype=np.uint8) for a in (x, x_scales, w1, w1_scales, w2, w2_scales)]
     x, xs, w1, s1, w2, s2 = arrs
     ids = np.ascontiguousarray(topk_ids, dtype=np.int32)
@@ -200,10 +206,11 @@ def fused_moe_mxfp8(x, x_scales, w1, w1_scales, w2, w2_scales, topk_ids, topk_we
     top_k = ids.shape[1]
     t, n = _tokens_arg(tokens, T)
     out = np.zeros((T, K), dtype=np.uint16)
+    f64 = np.zeros((T, K), dtype=np.float64) if unrounded else None
     _load().orc_fused_moe_mxfp8(_ptr(x), _ptr(xs), _ptr(w1), _ptr(s1), _ptr(w2), _ptr(s2), _ptr(ids),
                                 _ptr(tw), T, K, N, E, top_k, None if t is None else _ptr(t), n,
-                                _ptr(out), int(nthreads))
-    return out
+                                _ptr(out), None if f64 is None else _ptr(f64), int(nthreads))
+    return (out, f64) if unrounded else out
 
 
 def max_threads() -> int:

@@ -243,6 +243,13 @@ int orc_max_threads(void) {
 #endif
 }
 
+/* Both FFN routines can also hand back out before its final rounding
+ * (out_f64).  Reading: out is bf16 ([PFM] Shapes), and the last rounding is a
+ * decision that the GPU takes from an fp32 sum and the oracle from a double
+ * sum; the two can land one bf16 ulp apart, which for |out| >= 2.56 rms
+ * already exceeds a tolerance of 2e-2 rms.  Parity is therefore measured
+ * against the unrounded value.                                             */
+
 /* bf16 path ([PFM] intro and Shapes; [RFC] Background steps 2-5), one token
  * at a time, straight from the definition:
  *   for each route j of token t, e = topk_ids[t, j]:
@@ -254,7 +261,8 @@ int orc_max_threads(void) {
 void orc_fused_moe_bf16(const uint16_t* x, const uint16_t* w1, const uint16_t* w2,
                         const int32_t* topk_ids, const float* topk_weights,
                         int T, int K, int N, int E, int top_k,
-                        const int32_t* tokens, int n_tokens, uint16_t* out, int nthreads) {
+                        const int32_t* tokens, int n_tokens, uint16_t* out, double* out_f64,
+                        int nthreads) {
   const int I = N / 2;
   const int count = tokens ? n_tokens : T;
   set_threads(nthreads);
@@ -288,6 +296,8 @@ void orc_fused_moe_bf16(const uint16_t* x, const uint16_t* w1, const uint16_t* w
         }
       }
       for (int h = 0; h < K; ++h) out[(int64_t)t * K + h] = orc_double_to_bf16(acc[h]);
+      if (out_f64)
+        for (int h = 0; h < K; ++h) out_f64[(int64_t)t * K + h] = acc[h];
     }
     free(H); free(a); free(acc);
   }
@@ -305,7 +315,8 @@ void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
                          const uint8_t* w2, const uint8_t* w2_scales,
                          const int32_t* topk_ids, const float* topk_weights,
                          int T, int K, int N, int E, int top_k,
-                         const int32_t* tokens, int n_tokens, uint16_t* out, int nthreads) {
+                         const int32_t* tokens, int n_tokens, uint16_t* out, double* out_f64,
+                         int nthreads) {
   const int I = N / 2;
   const int KS = K / 32, IS = I / 32;
   const int count = tokens ? n_tokens : T;
@@ -353,6 +364,8 @@ void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
         }
       }
       for (int h = 0; h < K; ++h) out[(int64_t)t * K + h] = orc_double_to_bf16(acc[h]);
+      if (out_f64)
+        for (int h = 0; h < K; ++h) out_f64[(int64_t)t * K + h] = acc[h];
     }
     free(xd); free(H); free(af); free(aq); free(as); free(a); free(acc);
   }

@@ -46,11 +46,14 @@ void orc_unpack_scales_blocked(const uint8_t* in, uint8_t* out, int E, int MN, i
 
 /* ---- expert FFN -------------------------------------------------------- */
 /* out rows are written only for the tokens listed in `tokens` (n_tokens of
- * them, or all T when tokens == NULL).  nthreads <= 0 uses the OpenMP default. */
+ * them, or all T when tokens == NULL).  out_f64 (nullable, (T, K)) receives
+ * the same rows before the final rounding to bf16.  nthreads <= 0 uses the
+ * OpenMP default. */
 void orc_fused_moe_bf16(const uint16_t* x, const uint16_t* w1, const uint16_t* w2,
                         const int32_t* topk_ids, const float* topk_weights,
                         int T, int K, int N, int E, int top_k,
-                        const int32_t* tokens, int n_tokens, uint16_t* out, int nthreads);
+                        const int32_t* tokens, int n_tokens, uint16_t* out, double* out_f64,
+                        int nthreads);
 
 /* w1_scales / w2_scales are ROW-MAJOR here: (E, N, K/32) and (E, K, (N/2)/32). */
 void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
@@ -58,7 +61,8 @@ void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
                          const uint8_t* w2, const uint8_t* w2_scales,
                          const int32_t* topk_ids, const float* topk_weights,
                          int T, int K, int N, int E, int top_k,
-                         const int32_t* tokens, int n_tokens, uint16_t* out, int nthreads);
+                         const int32_t* tokens, int n_tokens, uint16_t* out, double* out_f64,
+                         int nthreads);
 
 /* Number of OpenMP threads a parallel region gets (for reporting). */
 int orc_max_threads(void);

@@ -171,3 +171,45 @@ def test_mxfp8_topk_weighted_and_zero():
         parts = parts + 0.5 * W.bf16_bits_to_f32(o).astype(np.float64)
     assert np.abs(both - parts).max() <= 2.0 ** -7 * np.abs(parts).max()
     assert not oracle.fused_moe_mxfp8(np.zeros_like(xq), xs, w1q, s1, w2q, s2, ids, tw).any()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "mxfp8"])
+def test_unrounded_output(dtype):
+    """out_f64 is out before its last rounding: rounding it gives out exactly,
+    and on the dense top-1 case it matches torch float64 to double precision
+    (up to the bf16 / mxfp8 rounding of the intermediate, done identically)."""
+    T, K, N, E = 24, 64, 128, 3
+    x, w1, w2, ids, tw = _small_inputs(T, K, N, E, 2, seed=99)
+    if dtype == "bf16":
+        out, f64 = oracle.fused_moe_bf16(x, w1, w2, ids, tw, unrounded=True)
+    else:
+        xq, xs = W.mx_quantize_inputs(W.bf16_bits_to_f32(x))
+        w1q, s1 = W.mx_quantize_inputs(W.bf16_bits_to_f32(w1))
+        w2q, s2 = W.mx_quantize_inputs(W.bf16_bits_to_f32(w2))
+        out, f64 = oracle.fused_moe_mxfp8(xq, xs, w1q, s1, w2q, s2, ids, tw, unrounded=True)
+    again = np.array([oracle.double_to_bf16(v) for v in f64.ravel()], dtype=np.uint16).reshape(out.shape)
+    np.testing.assert_array_equal(again, out)
+    assert np.abs(f64 - W.bf16_bits_to_f32(out)).max() <= 2.0 ** -8 * np.abs(f64).max()
+    # sampled rows, other rows untouched
+    sub = np.array([1, 7, 20], np.int32)
+    if dtype == "bf16":
+        _, part = oracle.fused_moe_bf16(x, w1, w2, ids, tw, tokens=sub, unrounded=True)
+    else:
+        _, part = oracle.fused_moe_mxfp8(xq, xs, w1q, s1, w2q, s2, ids, tw, tokens=sub, unrounded=True)
+    np.testing.assert_array_equal(part[sub], f64[sub])
+    assert not np.delete(part, sub, axis=0).any()
+
+
+def test_unrounded_dense_top1_matches_torch():
+    T, K, N, E = 30, 96, 64, 2
+    x, w1, w2, _, _ = _small_inputs(T, K, N, E, 1, seed=5)
+    ids = (np.arange(T) % E).astype(np.int32)[:, None]
+    _, f64 = oracle.fused_moe_bf16(x, w1, w2, ids, np.ones((T, 1), np.float32), unrounded=True)
+    xt = _bf16_to_t(x)
+    for e in range(E):
+        rows = np.nonzero(ids[:, 0] == e)[0]
+        h = F.linear(xt[rows], _bf16_to_t(w1[e]))
+        a = F.silu(h[:, : N // 2]) * h[:, N // 2:]
+        a_bits = np.array([oracle.double_to_bf16(v) for v in a.numpy().ravel()], np.uint16).reshape(a.shape)
+        ref = F.linear(torch.from_numpy(W.bf16_bits_to_f32(a_bits)).double(), _bf16_to_t(w2[e])).numpy()
+        np.testing.assert_allclose(f64[rows], ref, rtol=1e-9, atol=1e-12)
