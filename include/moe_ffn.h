@@ -1,0 +1,188 @@
+/*
+ * moe_ffn.h -- C ABI of the B200 (sm_100a) fused MoE expert-FFN forward.
+ *
+ * The operations and their arguments follow two pages:
+ *   [PFM] "Prime Flash MoE: Fused MoE Kernels for Blackwell" -- sections
+ *         intro (fused gate/up GEMM, SwiGLU consumed from the accumulator,
+ *         down GEMM, top-k weighted reduction; mxfp8 requant of the
+ *         intermediate), API, Shapes, Scale layout (mxfp8), Constraints.
+ *   [RFC] "[RFC] Fused W8A8 MoE megakernel on H20" -- sections Background
+ *         (the five local steps) and Design (planner: expert histogram,
+ *         prefix sums, row-to-token mapping; compute megakernel).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *     and row-major.  The library never allocates device memory per call and
+ *     never takes ownership of anything passed in.
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream) and
+ *     never synchronises with the host.
+ *   - Return value: MOE_OK (0) or a negative MOE_ERR_* code.  Arguments are
+ *     checked before anything is launched; on an argument error nothing is
+ *     launched and moe_last_error() describes the problem.  MOE_ERR_CUDA
+ *     reports a launch failure (the CUDA error string is in moe_last_error()).
+ *   - Faults found on the device (a bounded wait that ran out) are recorded
+ *     in a device status word read by moe_device_status().
+ *
+ * Readings of points the pages leave open (see the design notes):
+ *   - gate = rows [0, N/2) of w1[e], up = rows [N/2, N); act = silu(gate)*up.
+ *   - Inside an expert's segment of sorted_token_ids, route ids ascend.
+ *   - Unused capacity of sorted_token_ids and expert_ids is filled with -1.
+ *   - A topk_ids entry outside [0, E) routes nowhere: it gets no slot, and
+ *     contributes nothing to out.
+ */
+#ifndef MOE_FFN_H
+#define MOE_FFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Every entry point below is exported from libmoe_ffn.so. */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* same type as cudaStream_t */
+
+enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1, /* null pointer, negative or inconsistent size */
+  MOE_ERR_UNSUPPORTED = -2, /* a shape outside the supported constraints   */
+  MOE_ERR_ALIGNMENT = -3,   /* a pointer not aligned as the kernel needs   */
+  MOE_ERR_WORKSPACE = -4,   /* workspace missing or smaller than required  */
+  MOE_ERR_CUDA = -5,        /* a CUDA runtime / driver call failed         */
+  MOE_ERR_TIMEOUT = -6      /* a device-side bounded wait ran out          */
+};
+
+enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_MXFP8 = 1 };
+
+/* Message describing the last error returned on the calling host thread. */
+MOE_API const char* moe_last_error(void);
+
+/* Waits for `stream`, then returns MOE_OK, or MOE_ERR_TIMEOUT if a kernel of
+ * this library running on the current device gave up a bounded wait since the
+ * previous call; the status word is cleared. */
+MOE_API int moe_device_status(moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * moe_align -- the routing planner.
+ * [RFC] Design: count routed tokens per expert (histogram), prefix sums over
+ * the counts, row-to-token mapping.  [PFM] API / Shapes: sorted_token_ids
+ * holds flattened token*top_k+route ids grouped by expert, each group padded
+ * to a multiple of block_m with -1; expert_ids gives the expert of every
+ * block_m block; num_tokens_post_padded the padded total.
+ *
+ *   topk_ids            (T, top_k) int32, device, read only.
+ *   sorted_token_ids    capacity int32, device, written in full: ids of the
+ *                       routes to expert 0 (ascending), -1 up to a multiple
+ *                       of block_m, then expert 1, ...; -1 from
+ *                       num_tokens_post_padded to capacity.
+ *   expert_ids          ceil(capacity / block_m) int32, device, written in
+ *                       full: expert of block b for b < ntpp / block_m,
+ *                       else -1.  Experts with no routes get no block.
+ *   num_tokens_post_padded  one int32, device: sum over experts of
+ *                       ceil(count / block_m) * block_m.
+ *   capacity            must be >= moe_align_capacity(T, top_k, E, block_m).
+ * Constraints: T >= 0, top_k >= 1, 1 <= E <= 1024, block_m in {16, 32, 64,
+ * 128}; T * top_k + E * (block_m - 1) < 2^31.  T = 0 is allowed.
+ * ---------------------------------------------------------------------- */
+MOE_API int64_t moe_align_capacity(int T, int top_k, int E, int block_m);
+MOE_API int moe_align(const int32_t* topk_ids, int T, int top_k, int E, int block_m,
+              int32_t* sorted_token_ids, int32_t* expert_ids, int32_t* num_tokens_post_padded,
+              int64_t capacity, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * pack_scales_blocked -- [PFM] Scale layout (mxfp8): weight scales (one e8m0
+ * byte per 32 along K) reordered into a sequence of 512-byte tiles, each
+ * covering 128 rows (MN) x 128 K (4 scale bytes).  Tile (e, mt, kt) starts at
+ * byte ((e * MT + mt) * KT + kt) * 512 with MT = ceil(MN/128),
+ * KT = ceil(KS/4); inside a tile, row r and scale column c sit at byte
+ * (r % 32) * 16 + (r / 32) * 4 + c (the 128 x 4 scale-factor arrangement the
+ * Blackwell block-scaled MMA reads).  Bytes outside (MN, KS) are written 0.
+ *
+ *   in   (E, MN, KS) uint8, row major, device.
+ *   out  pack_scales_blocked_bytes(E, MN, KS) bytes, device, written in full.
+ * Run once at weight-load time, not per step.
+ * ---------------------------------------------------------------------- */
+MOE_API int64_t pack_scales_blocked_bytes(int E, int MN, int KS);
+MOE_API int pack_scales_blocked(const uint8_t* in, uint8_t* out, int E, int MN, int KS,
+                        moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Workspace.  fused_moe_* need caller-owned device scratch of at least
+ * moe_workspace_bytes(...) bytes, 256-byte aligned.  It holds the SwiGLU
+ * intermediate of every routed row (written once, read once by the down
+ * projection), the weighted down-projection rows of every route, and one
+ * flag per route.  Its contents need no initialisation and are garbage
+ * afterwards; two calls that overlap in time must not share it.
+ * ---------------------------------------------------------------------- */
+MOE_API int64_t moe_workspace_bytes(int dtype, int T, int K, int N, int E, int top_k, int block_m);
+
+/* Optional tuning knobs; pass NULL for the defaults (0 / NULL in a field
+ * also means "default"). */
+typedef struct moe_tuning {
+  int stages;   /* shared-memory pipeline depth of the GEMM phases        */
+  int num_ctas; /* persistent CTAs per phase (default: one per SM)        */
+  /* Timing hook: if non-NULL, four caller-created cudaEvent_t handles that
+   * are recorded on `stream` before the gate/up phase, between it and the
+   * down phase, between the down phase and the reduction, and after the
+   * reduction. */
+  void* const* phase_events;
+} moe_tuning;
+
+/* ------------------------------------------------------------------------
+ * fused_moe_bf16 -- [PFM] intro / API / Shapes, bf16 path; [RFC] Background
+ * steps 2-5.  For every routed row (token t, route j, expert e):
+ *   H   = w1[e] . x[t]                  (N values, fp32 accumulation)
+ *   a_i = bf16( silu(H_i) * H_{N/2+i} )  i < N/2
+ *   Y   = w2[e] . a                      (K values, fp32 accumulation)
+ * and out[t] = bf16( sum_j topk_weights[t, j] * Y_(t, j) ).
+ *
+ *   x             (T, K) bf16            w1 (E, N, K) bf16
+ *   w2            (E, K, N/2) bf16       out (T, K) bf16, overwritten
+ *   topk_weights  (T, top_k) fp32
+ *   sorted_token_ids / expert_ids / num_tokens_post_padded: moe_align's
+ *                 outputs for the same (T, top_k, E, block_m, capacity).
+ * Constraints: K % 128 == 0, N % 16 == 0, N >= 16, block_m in {16, 32, 64,
+ * 128}; every pointer 16-byte aligned, workspace 256-byte aligned.
+ * ---------------------------------------------------------------------- */
+MOE_API int fused_moe_bf16(const void* x, const void* w1, const void* w2,
+                   const int32_t* sorted_token_ids, const int32_t* expert_ids,
+                   const int32_t* num_tokens_post_padded, const float* topk_weights, void* out,
+                   int T, int K, int N, int E, int top_k, int block_m, int64_t capacity,
+                   void* workspace, int64_t workspace_bytes, const moe_tuning* tune,
+                   moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * fused_moe_mxfp8 -- [PFM] intro / API / Scale layout (mxfp8), mxfp8 path:
+ * e4m3 values with one e8m0 scale per 32 along the contraction dimension on
+ * both operands of both GEMMs, fp32 accumulation; the SwiGLU intermediate is
+ * requantised on chip (per routed row, per 32 along N/2: amax, e8m0 scale
+ * 2^(floor(log2 amax) - 8), e4m3 round-to-nearest-even with saturation)
+ * before the down GEMM; bf16 out.
+ *
+ *   x_e4m3 (T, K) u8            x_scales (T, K/32) u8 e8m0, ROW MAJOR
+ *   w1_e4m3 (E, N, K) u8        w1_scales_blocked = pack_scales_blocked of
+ *                               the (E, N, K/32) scales
+ *   w2_e4m3 (E, K, N/2) u8      w2_scales_blocked = pack_scales_blocked of
+ *                               the (E, K, N/64) scales
+ *   other arguments as fused_moe_bf16.
+ * Constraints: K % 256 == 0, N % 256 == 0, block_m in {16, 32, 64, 128}.
+ * ---------------------------------------------------------------------- */
+MOE_API int fused_moe_mxfp8(const uint8_t* x_e4m3, const uint8_t* x_scales, const uint8_t* w1_e4m3,
+                    const uint8_t* w1_scales_blocked, const uint8_t* w2_e4m3,
+                    const uint8_t* w2_scales_blocked, const int32_t* sorted_token_ids,
+                    const int32_t* expert_ids, const int32_t* num_tokens_post_padded,
+                    const float* topk_weights, void* out, int T, int K, int N, int E, int top_k,
+                    int block_m, int64_t capacity, void* workspace, int64_t workspace_bytes,
+                    const moe_tuning* tune, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_FFN_H */

@@ -1,0 +1,264 @@
+"""Python binding of the B200 fused MoE expert-FFN forward (``libmoe_ffn.so``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/moe_ffn.h``.  PyTorch supplies
+device memory and streams.  There is no CPU or PyTorch fallback: if the
+library cannot be built or loaded, every call raises.
+
+Entry points (same names as the C ABI):
+
+* ``moe_align`` -- routing planner: expert histogram, prefix sums over counts
+  padded to ``block_m``, and the row-to-token map ("[RFC] Fused W8A8 MoE
+  megakernel on H20", Design; "Prime Flash MoE: Fused MoE Kernels for
+  Blackwell", API / Shapes).
+* ``fused_moe_bf16`` / ``fused_moe_mxfp8`` -- gather, gate/up GEMM, SwiGLU
+  (mxfp8: on-chip requant of the intermediate), down GEMM and the top-k
+  weighted reduction into ``out`` ("Prime Flash MoE", intro / API / Shapes).
+* ``pack_scales_blocked`` -- weight scales into 512-byte tiles of
+  128 MN x 128 K ("Prime Flash MoE", Scale layout (mxfp8)).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+from . import _build
+
+__all__ = [
+    "MoeError", "load", "moe_align", "moe_align_capacity", "fused_moe_bf16", "fused_moe_mxfp8",
+    "pack_scales_blocked", "pack_scales_blocked_bytes", "moe_workspace_bytes", "moe_device_status",
+    "Tuning", "DTYPE_BF16", "DTYPE_MXFP8", "LIB_PATH",
+]
+
+DTYPE_BF16 = 0
+DTYPE_MXFP8 = 1
+LIB_PATH = _build.LIB
+
+_ERRORS = {-1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_ALIGNMENT",
+           -4: "MOE_ERR_WORKSPACE", -5: "MOE_ERR_CUDA", -6: "MOE_ERR_TIMEOUT"}
+
+
+class MoeError(RuntimeError):
+    """A C-ABI call returned a negative status."""
+
+    def __init__(self, code: int, message: str):
+        self.code = int(code)
+        self.name = _ERRORS.get(self.code, f"status {code}")
+        super().__init__(f"{self.name}: {message}")
+
+
+class Tuning(ctypes.Structure):
+    """``moe_tuning``: 0 in a field keeps the library's default."""
+    _fields_ = [("stages", ctypes.c_int), ("num_ctas", ctypes.c_int),
+                ("phase_events", ctypes.POINTER(ctypes.c_void_p))]
+
+    @staticmethod
+    def with_events(events, stages: int = 0, num_ctas: int = 0) -> "Tuning":
+        """Tuning whose timing hook records the four given torch.cuda.Event objects."""
+        for e in events:
+            e.record()  # forces creation of the underlying cudaEvent_t
+        arr = (ctypes.c_void_p * 4)(*[e.cuda_event for e in events])
+        t = Tuning(stages, num_ctas, ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)))
+        t._keep = arr
+        return t
+
+
+_lock = threading.Lock()
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+
+_SIGS = {
+    "moe_last_error": ([], ctypes.c_char_p),
+    "moe_device_status": ([_P], _I),
+    "moe_align_capacity": ([_I, _I, _I, _I], _I64),
+    "moe_align": ([_P, _I, _I, _I, _I, _P, _P, _P, _I64, _P], _I),
+    "pack_scales_blocked_bytes": ([_I, _I, _I], _I64),
+    "pack_scales_blocked": ([_P, _P, _I, _I, _I, _P], _I),
+    "moe_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I], _I64),
+    "fused_moe_bf16": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _I64, _P, _P], _I),
+    "fused_moe_mxfp8": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _I64,
+                         _P, _P], _I),
+}
+
+
+def load(build_if_stale: bool = True) -> ctypes.CDLL:
+    """Loads libmoe_ffn.so (compiling it first if a source is newer)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if build_if_stale and _build.stale():
+            try:
+                _build.build()
+            except Exception as exc:  # no toolchain: use the library that is there, if any
+                if not os.path.exists(_build.LIB):
+                    raise ImportError(f"libmoe_ffn.so is missing and could not be built: {exc}") from exc
+        if not os.path.exists(_build.LIB):
+            raise ImportError(f"libmoe_ffn.so not found at {_build.LIB}; run __graft_entry__.build()")
+        lib = ctypes.CDLL(_build.LIB)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+        return lib
+
+
+def _check(rc: int):
+    if rc != 0:
+        msg = load().moe_last_error()
+        raise MoeError(rc, msg.decode() if msg else "")
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t, name, dtypes, device=True):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+
+
+# ---------------------------------------------------------------- sizes
+def moe_align_capacity(T: int, top_k: int, E: int, block_m: int) -> int:
+    return int(load().moe_align_capacity(T, top_k, E, block_m))
+
+
+def pack_scales_blocked_bytes(E: int, MN: int, KS: int) -> int:
+    return int(load().pack_scales_blocked_bytes(E, MN, KS))
+
+
+def moe_workspace_bytes(dtype: int, T: int, K: int, N: int, E: int, top_k: int, block_m: int) -> int:
+    n = int(load().moe_workspace_bytes(dtype, T, K, N, E, top_k, block_m))
+    if n < 0:
+        raise MoeError(-1, "moe_workspace_bytes: invalid arguments")
+    return n
+
+
+# ---------------------------------------------------------------- calls
+def moe_align(topk_ids, E: int, block_m: int, sorted_token_ids=None, expert_ids=None,
+              num_tokens_post_padded=None, stream=None):
+    """Routing planner.  Returns (sorted_token_ids, expert_ids, num_tokens_post_padded)."""
+    import torch
+
+    _need(topk_ids, "topk_ids", (torch.int32,))
+    T, top_k = topk_ids.shape
+    cap = moe_align_capacity(T, top_k, E, block_m)
+    if cap < 0:
+        raise MoeError(-1, "moe_align: invalid sizes")
+    dev = topk_ids.device
+    if sorted_token_ids is None:
+        sorted_token_ids = torch.empty(cap, dtype=torch.int32, device=dev)
+    if expert_ids is None:
+        expert_ids = torch.empty((sorted_token_ids.numel() + block_m - 1) // block_m, dtype=torch.int32,
+                                 device=dev)
+    if num_tokens_post_padded is None:
+        num_tokens_post_padded = torch.empty(1, dtype=torch.int32, device=dev)
+    for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
+                 (num_tokens_post_padded, "num_tokens_post_padded")):
+        _need(t, n, (torch.int32,))
+    if expert_ids.numel() < (sorted_token_ids.numel() + block_m - 1) // block_m:
+        raise ValueError("expert_ids must hold ceil(capacity / block_m) entries")
+    _check(load().moe_align(_ptr(topk_ids), T, top_k, E, block_m, _ptr(sorted_token_ids), _ptr(expert_ids),
+                            _ptr(num_tokens_post_padded), sorted_token_ids.numel(), _stream(stream)))
+    return sorted_token_ids, expert_ids, num_tokens_post_padded
+
+
+def pack_scales_blocked(scales, out=None, stream=None):
+    """(E, MN, KS) uint8 e8m0 scales, row major -> blocked 512-byte tiles (uint8, flat)."""
+    import torch
+
+    _need(scales, "scales", (torch.uint8,))
+    E, MN, KS = scales.shape
+    n = pack_scales_blocked_bytes(E, MN, KS)
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=scales.device)
+    _need(out, "out", (torch.uint8,))
+    if out.numel() < n:
+        raise ValueError(f"out must hold {n} bytes")
+    _check(load().pack_scales_blocked(_ptr(scales), _ptr(out), E, MN, KS, _stream(stream)))
+    return out
+
+
+def _workspace(dtype, T, K, N, E, top_k, block_m, workspace, device):
+    import torch
+
+    need = moe_workspace_bytes(dtype, T, K, N, E, top_k, block_m)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    _need(workspace, "workspace", (torch.uint8,))
+    return workspace
+
+
+def fused_moe_bf16(x, w1, w2, sorted_token_ids, expert_ids, num_tokens_post_padded, topk_weights, out,
+                   block_m: int, workspace=None, tune: Tuning | None = None, stream=None):
+    """bf16 path.  x (T,K), w1 (E,N,K), w2 (E,K,N/2) bf16; topk_weights (T,top_k) fp32; out (T,K) bf16."""
+    import torch
+
+    for t, n in ((x, "x"), (w1, "w1"), (w2, "w2"), (out, "out")):
+        _need(t, n, (torch.bfloat16,))
+    _need(topk_weights, "topk_weights", (torch.float32,))
+    for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
+                 (num_tokens_post_padded, "num_tokens_post_padded")):
+        _need(t, n, (torch.int32,))
+    T, K = x.shape
+    E, N, _ = w1.shape
+    top_k = topk_weights.shape[1]
+    ws = _workspace(DTYPE_BF16, T, K, N, E, top_k, block_m, workspace, x.device)
+    _check(load().fused_moe_bf16(
+        _ptr(x), _ptr(w1), _ptr(w2), _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded),
+        _ptr(topk_weights), _ptr(out), T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws), ws.numel(),
+        None if tune is None else ctypes.byref(tune), _stream(stream)))
+    return out
+
+
+def fused_moe_mxfp8(x, x_scales, w1, w1_scales_blocked, w2, w2_scales_blocked, sorted_token_ids, expert_ids,
+                    num_tokens_post_padded, topk_weights, out, block_m: int, workspace=None,
+                    tune: Tuning | None = None, stream=None):
+    """mxfp8 path.  e4m3 codes as uint8 (or float8_e4m3fn), e8m0 scales as uint8; out (T,K) bf16."""
+    import torch
+
+    u8 = (torch.uint8, torch.float8_e4m3fn)
+    for t, n in ((x, "x"), (w1, "w1"), (w2, "w2")):
+        _need(t, n, u8)
+    for t, n in ((x_scales, "x_scales"), (w1_scales_blocked, "w1_scales_blocked"),
+                 (w2_scales_blocked, "w2_scales_blocked")):
+        _need(t, n, (torch.uint8,))
+    _need(out, "out", (torch.bfloat16,))
+    _need(topk_weights, "topk_weights", (torch.float32,))
+    for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
+                 (num_tokens_post_padded, "num_tokens_post_padded")):
+        _need(t, n, (torch.int32,))
+    T, K = x.shape
+    E, N, _ = w1.shape
+    top_k = topk_weights.shape[1]
+    ws = _workspace(DTYPE_MXFP8, T, K, N, E, top_k, block_m, workspace, x.device)
+    _check(load().fused_moe_mxfp8(
+        _ptr(x), _ptr(x_scales), _ptr(w1), _ptr(w1_scales_blocked), _ptr(w2), _ptr(w2_scales_blocked),
+        _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(topk_weights), _ptr(out),
+        T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws), ws.numel(),
+        None if tune is None else ctypes.byref(tune), _stream(stream)))
+    return out
+
+
+def moe_device_status(stream=None):
+    """Waits for the stream; raises MoeError(MOE_ERR_TIMEOUT) if a device-side wait gave up."""
+    _check(load().moe_device_status(_stream(stream)))

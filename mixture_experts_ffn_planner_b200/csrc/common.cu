@@ -1,0 +1,37 @@
+// Error reporting and device queries shared by every entry point.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "internal.h"
+
+namespace moe {
+
+static thread_local char g_last_error[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(const char* what, cudaError_t err) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(err));
+  return MOE_ERR_CUDA;
+}
+
+int sm_count() {
+  static int cached[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < kMaxDevices && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < kMaxDevices) cached[dev] = n;
+  return n;
+}
+
+}  // namespace moe
+
+extern "C" const char* moe_last_error(void) { return moe::g_last_error; }

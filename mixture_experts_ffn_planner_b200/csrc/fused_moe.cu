@@ -1,0 +1,939 @@
+// Fused MoE expert-FFN forward for sm_100a (bf16 and mxfp8 paths).
+//
+// What is computed -- "Prime Flash MoE: Fused MoE Kernels for Blackwell",
+// intro / API / Shapes, and "[RFC] Fused W8A8 MoE megakernel on H20",
+// Background: for every routed row (token t, route j, expert e) the gate/up
+// GEMM H = w1[e] x[t], SwiGLU a = silu(H[:N/2]) * H[N/2:] taken straight from
+// the accumulator (never stored as the 2H-wide tensor), on the mxfp8 path a
+// requantisation of a to e4m3 + e8m0 per 32 on chip, the down GEMM
+// Y = w2[e] a, and the top-k weighted reduction out[t] = sum_j w[t,j] Y.
+//
+// How (sm_100a):
+//   phase 1  persistent kernel, one CTA per SM.  A work unit is (planner block
+//            b, intermediate tile j of 128 columns).  The expert's weights are
+//            the 128-row A operand of tcgen05.mma (gate rows and up rows, one
+//            MMA each), the block's gathered token rows are the B operand, so
+//            the MMA's N is the number of routed rows rounded up to 16 and the
+//            accumulators live in TMEM as [weight row (lane)] x [token
+//            (column)].  Gate row i and up row i land in the same TMEM lane,
+//            so one thread computes silu(g)*u for its intermediate column and
+//            (mxfp8) takes the 32-wide amax with one warp redux.  The
+//            intermediate is written once to an L2-resident workspace.
+//            Warp roles: 0 TMA producer (weight tiles, weight scale tiles),
+//            1 MMA issuer, 2-5 token gather (cp.async, 128-byte swizzle, token
+//            scales), 6-9 epilogue.
+//   phase 2  persistent kernel, unit = (block b, 128 output features).  A =
+//            w2[e] rows, B = the block's intermediate rows (TMA), D in TMEM;
+//            the epilogue scales by the routing weight and writes one fp32 row
+//            per route.
+//   combine  out[t] = bf16(sum over the token's routes, in route order), a
+//            deterministic HBM-bound pass.
+// The weight tile of a unit is streamed once through a multi-stage shared
+// memory ring by TMA; the weights are the dominant HBM traffic.
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+__device__ int g_moe_status = 0;
+
+constexpr int kTile = 128;        // weight rows per MMA (M) and features per unit
+constexpr int kRowBytes = 128;    // bytes of one operand row per pipeline stage
+constexpr int kSfTileBytes = 512; // one blocked scale tile: 128 rows x 4 scales
+constexpr int kSmemLimit = 232448;  // 227 KB of dynamic shared memory per CTA
+
+// TMEM column map
+constexpr uint32_t kP1SfCol = 256;  // mxfp8 scale factors (12 columns) in phase 1
+constexpr uint32_t kP2SfCol = 256;  // mxfp8 scale factors (8 columns) in phase 2
+
+constexpr int kP1Threads = 320;  // 10 warps
+constexpr int kP1GatherWarps = 4;
+constexpr int kP2Threads = 192;  // 6 warps
+
+struct P1Params {
+  const uint8_t* x;         // (T, K) bf16 or e4m3
+  const uint8_t* x_sf;      // (T, K/32) e8m0, row major (mxfp8)
+  const uint8_t* w1_sf;     // blocked scales of w1 (mxfp8)
+  const int32_t* sorted_ids;
+  const int32_t* expert_ids;
+  const int32_t* ntpp;
+  uint8_t* act;             // (cap_rows, I) bf16 or e4m3
+  uint8_t* act_sf;          // blocked scales of act, one tile row per block (mxfp8)
+  int32_t* flags;           // one per route, cleared here
+  int* status;
+  int K, N, I, E, top_k, bm, R;
+  int max_blocks;           // workspace rows / bm
+  int n_jt;                 // ceil(I / 128)
+  int stages, stage_bytes;
+};
+
+struct P2Params {
+  const uint8_t* w2_sf;     // blocked scales of w2 (mxfp8)
+  const uint8_t* act_sf;
+  const int32_t* sorted_ids;
+  const int32_t* expert_ids;
+  const int32_t* ntpp;
+  const float* topk_w;
+  float* yw;                // (R, K) weighted down-projection rows
+  int32_t* flags;
+  int* status;
+  int K, I, E, top_k, bm, R;
+  int max_blocks;
+  int n_ht;                 // K / 128
+  int n_kc;                 // K-chunks of the down GEMM
+  int stages, stage_bytes;
+};
+
+// Per-unit facts every warp role derives the same way (warp-collective).
+struct BlockInfo {
+  int e;            // expert of the block
+  int nend;         // 1 + index of the last routed row in the block (0: none)
+  int n16;          // MMA N: nend rounded up to 16
+  uint32_t vm[4];   // routed-row mask, rows 32q .. 32q+31
+};
+
+__device__ __forceinline__ BlockInfo block_info(const int32_t* sorted_ids, const int32_t* expert_ids, int b,
+                                                int bm, int R, int E) {
+  BlockInfo bi;
+  const int lane = static_cast<int>(lane_id());
+  bi.e = __ldg(expert_ids + b);
+  bi.nend = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int r = 32 * q + lane;
+    bool v = false;
+    if (r < bm) {
+      const int id = __ldg(sorted_ids + static_cast<int64_t>(b) * bm + r);
+      v = id >= 0 && id < R;
+    }
+    bi.vm[q] = __ballot_sync(0xffffffffu, v);
+    if (bi.vm[q]) bi.nend = 32 * q + 32 - __clz(static_cast<int>(bi.vm[q]));
+  }
+  if (bi.e < 0 || bi.e >= E) bi.nend = 0;
+  bi.n16 = (bi.nend + 15) & ~15;
+  return bi;
+}
+
+__device__ __forceinline__ bool row_valid(const BlockInfo& bi, int c) {
+  return (bi.vm[c >> 5] >> (c & 31)) & 1u;
+}
+
+__device__ __forceinline__ int num_blocks(const int32_t* ntpp, int bm, int max_blocks) {
+  const int n = __ldg(ntpp) / bm;
+  return n < 0 ? 0 : (n > max_blocks ? max_blocks : n);
+}
+
+// After a wait gave up, copies and MMAs issued before the abort may still be
+// landing in shared memory / TMEM.  They finish within microseconds; wait a
+// bounded 100 us before the CTA releases its TMEM and exits.
+__device__ __forceinline__ void drain_after_abort() {
+  const unsigned long long t0 = globaltimer();
+  while (globaltimer() - t0 < 100000ull) __nanosleep(1000);
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  const uint32_t a = smem_u32(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+// ========================================================================
+// phase 1: gate/up GEMM + SwiGLU (+ mxfp8 requant) -> intermediate
+// ========================================================================
+template <bool kFp8>
+__global__ void __launch_bounds__(kP1Threads, 1)
+    moe_p1_kernel(const __grid_constant__ CUtensorMap tm_w1, const __grid_constant__ P1Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const int S = p.stages;
+  uint8_t* ctrl = smem + static_cast<size_t>(S) * p.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sm + 1);
+  int32_t* tok_tab = reinterpret_cast<int32_t*>(tmem_base_sm + 4);  // [kP1GatherWarps][128]
+
+  constexpr int kNumAcc = kFp8 ? 1 : 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // clear the route flags (phase 2 sets them); nothing reads them in this phase
+  for (int i = blockIdx.x * kP1Threads + threadIdx.x; i < p.R; i += gridDim.x * kP1Threads) p.flags[i] = 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1 + 32);  // TMA producer + the 32 lanes of one gather warp
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_w1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_sm, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_base_sm;
+
+  const int n_blocks = num_blocks(p.ntpp, p.bm, p.max_blocks);
+  const int n_units = n_blocks * p.n_jt;
+  constexpr int kKC = kFp8 ? 128 : 64;  // K elements per stage (128 bytes per row)
+  const int n_kc = p.K / kKC;
+  const int esize = kFp8 ? 1 : 2;
+
+  auto stage_ptr = [&](int s) { return smem + static_cast<size_t>(s) * p.stage_bytes; };
+  // stage layout: [A gate 16K][A up 16K][B bm*128][SFA gate 512][SFA up 512][SFB 512]
+  const int off_b = 2 * kTile * kRowBytes;
+  const int off_sf = off_b + p.bm * kRowBytes;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    const uint64_t pol = policy_evict_first();
+    const uint32_t tx = 2 * kTile * kRowBytes + (kFp8 ? 2 * kSfTileBytes : 0);
+    const int MT1 = p.N / kTile, KT1 = p.K / 128;
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int b = u / p.n_jt, j = u - (u / p.n_jt) * p.n_jt;
+      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      if (bi.nend == 0) continue;
+      const int gate_row = bi.e * p.N + j * kTile;
+      const int up_row = bi.e * p.N + p.I + j * kTile;
+      for (int kc = 0; kc < n_kc; ++kc) {
+        if (lane == 0) {
+          ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
+          if (ok) {
+            uint8_t* st = stage_ptr(s);
+            mbar_arrive_expect_tx(&full[s], tx);
+            tma_load_2d(st, &tm_w1, &full[s], kc * kKC, gate_row, pol);
+            tma_load_2d(st + kTile * kRowBytes, &tm_w1, &full[s], kc * kKC, up_row, pol);
+            if (kFp8) {
+              const uint8_t* sfg = p.w1_sf + ((static_cast<int64_t>(bi.e) * MT1 + j) * KT1 + kc) * kSfTileBytes;
+              const uint8_t* sfu =
+                  p.w1_sf + ((static_cast<int64_t>(bi.e) * MT1 + p.I / kTile + j) * KT1 + kc) * kSfTileBytes;
+              bulk_load(st + off_sf, sfg, kSfTileBytes, &full[s]);
+              bulk_load(st + off_sf + kSfTileBytes, sfu, kSfTileBytes, &full[s]);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (++s == S) { s = 0; ph ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    int s = 0;
+    uint32_t ph = 0;
+    int acc_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int b = u / p.n_jt;
+      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      if (bi.nend == 0) continue;
+      const int buf = acc_it % kNumAcc;
+      const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
+      if (lane == 0) ok = mbar_wait(&acc_empty[buf], acc_ph ^ 1u, abort_flag, p.status);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t d_gate = tbase + static_cast<uint32_t>(buf) * 256u;
+      const uint32_t d_up = d_gate + 128u;
+      for (int kc = 0; kc < n_kc; ++kc) {
+        if (lane == 0) {
+          ok = mbar_wait(&full[s], ph, abort_flag, p.status);
+          if (ok) {
+            tc_fence_after();
+            uint8_t* st = stage_ptr(s);
+            const uint64_t ag = sdesc_sw128(smem_u32(st));
+            const uint64_t au = sdesc_sw128(smem_u32(st + kTile * kRowBytes));
+            const uint64_t bd = sdesc_sw128(smem_u32(st + off_b));
+            if (kFp8) {
+              tc_cp_32x128b_x4(tbase + kP1SfCol + 0, sdesc_sf(smem_u32(st + off_sf)));
+              tc_cp_32x128b_x4(tbase + kP1SfCol + 4, sdesc_sf(smem_u32(st + off_sf + kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + kP1SfCol + 8, sdesc_sf(smem_u32(st + off_sf + 2 * kSfTileBytes)));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (kc | kk) != 0;
+              const uint64_t step = static_cast<uint64_t>(2 * kk);  // 32 bytes along K
+              if (kFp8) {
+                const uint32_t id = idesc_mxf8(kTile, bi.n16, kk, kk);
+                const uint32_t sfid = static_cast<uint32_t>(kk) << 30;
+                const uint32_t sfb = (tbase + kP1SfCol + 8) | sfid;
+                mma_mxf8(d_gate, ag + step, bd + step, id, (tbase + kP1SfCol + 0) | sfid, sfb, acc);
+                mma_mxf8(d_up, au + step, bd + step, id, (tbase + kP1SfCol + 4) | sfid, sfb, acc);
+              } else {
+                const uint32_t id = idesc_bf16(kTile, bi.n16);
+                mma_f16(d_gate, ag + step, bd + step, id, acc);
+                mma_f16(d_up, au + step, bd + step, id, acc);
+              }
+            }
+            tc_commit(&empty[s]);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (++s == S) { s = 0; ph ^= 1u; }
+      }
+      if (ok && lane == 0) tc_commit(&acc_full[buf]);
+      ++acc_it;
+    }
+  } else if (warp < 2 + kP1GatherWarps) {
+    // ------------------------------------------------ token gather
+    const int g = warp - 2;
+    int32_t* tok = tok_tab + g * 128;
+    // Gather warp g owns the stages s with s % kP1GatherWarps == g and fills
+    // every use of them in order, so its wait on empty[s] is never more than
+    // one phase behind the barrier (a parity wait cannot tell phase n from
+    // phase n + 2).
+    const int KS = p.K / 32;
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int b = u / p.n_jt;
+      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      if (bi.nend == 0) continue;
+      bool tok_ready = false;
+      for (int kc = 0; kc < n_kc; ++kc) {
+        if (s % kP1GatherWarps == g) {
+          if (!tok_ready) {
+            __syncwarp();
+            for (int r = lane; r < bi.n16; r += 32) {
+              const int id = __ldg(p.sorted_ids + static_cast<int64_t>(b) * p.bm + r);
+              tok[r] = row_valid(bi, r) ? id / p.top_k : -1;
+            }
+            __syncwarp();
+            tok_ready = true;
+          }
+          if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          uint8_t* st = stage_ptr(s);
+          const uint32_t bsm = smem_u32(st + off_b);
+          for (int idx = lane; idx < bi.n16 * 8; idx += 32) {
+            const int r = idx >> 3, q = idx & 7;
+            const uint32_t dst = bsm + r * kRowBytes + ((q ^ (r & 7)) << 4);
+            const int t = tok[r];
+            if (t >= 0) {
+              cp_async_16(dst, p.x + (static_cast<int64_t>(t) * p.K * esize + kc * kRowBytes + q * 16));
+            } else {
+              asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
+            }
+          }
+          if (kFp8) {
+            uint8_t* sfb = st + off_sf + 2 * kSfTileBytes;
+            for (int r = lane; r < bi.n16; r += 32) {
+              const int t = tok[r];
+              uint32_t v = 0;
+              if (t >= 0) v = __ldg(reinterpret_cast<const uint32_t*>(p.x_sf + static_cast<int64_t>(t) * KS) + kc);
+              *reinterpret_cast<uint32_t*>(sfb + (r & 31) * 16 + (r >> 5) * 4) = v;
+            }
+          }
+          cp_async_commit();
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+          mbar_arrive(&full[s]);
+        }
+        if (++s == S) { s = 0; ph ^= 1u; }
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quadrant of this warp
+    int acc_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int b = u / p.n_jt, j = u - (u / p.n_jt) * p.n_jt;
+      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      if (bi.nend == 0) continue;
+      const int buf = acc_it % kNumAcc;
+      const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
+      ok = mbar_wait(&acc_full[buf], acc_ph, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 256u;
+      const int icol = j * kTile + 32 * q + lane;
+      const int64_t row0 = static_cast<int64_t>(b) * p.bm;
+      for (int c0 = 0; c0 < bi.nend; c0 += 16) {
+        uint32_t gr[16], ur[16];
+        tmem_ld16(tacc + c0, gr);
+        tmem_ld16(tacc + 128 + c0, ur);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = c0 + i;
+          const float a = silu_f32(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
+          if (kFp8) {
+            const uint32_t amax_bits = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(a)));
+            int sc = static_cast<int>((amax_bits >> 23) & 0xFFu) - 127 - 8;
+            sc = sc < -127 ? -127 : (sc > 127 ? 127 : sc);
+            const float inv = __uint_as_float(static_cast<uint32_t>(127 - sc) << 23);
+            if (row_valid(bi, c)) {
+              p.act[(row0 + c) * p.I + icol] = static_cast<uint8_t>(cvt_e4m3x2(a * inv, 0.0f) & 0xFFu);
+              if (lane == 0)
+                p.act_sf[(static_cast<int64_t>(b) * p.n_jt + j) * kSfTileBytes + (c & 31) * 16 + (c >> 5) * 4 + q] =
+                    static_cast<uint8_t>(sc + 127);
+            }
+          } else {
+            if (row_valid(bi, c) && icol < p.I)
+              reinterpret_cast<__nv_bfloat16*>(p.act)[(row0 + c) * p.I + icol] = __float2bfloat16_rn(a);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      ++acc_it;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) drain_after_abort();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ========================================================================
+// phase 2: down GEMM + routing weight -> one fp32 row per route
+// ========================================================================
+template <bool kFp8>
+__global__ void __launch_bounds__(kP2Threads, 1)
+    moe_p2_kernel(const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_act,
+                  const __grid_constant__ P2Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const int S = p.stages;
+  uint8_t* ctrl = smem + static_cast<size_t>(S) * p.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(ctrl);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sm + 1);
+
+  constexpr int kNumAcc = 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_w2);
+    prefetch_tmap(&tm_act);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_sm, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_base_sm;
+
+  const int n_blocks = num_blocks(p.ntpp, p.bm, p.max_blocks);
+  const int n_units = n_blocks * p.n_ht;
+  constexpr int kKC = kFp8 ? 128 : 64;
+  auto stage_ptr = [&](int s) { return smem + static_cast<size_t>(s) * p.stage_bytes; };
+  // stage layout: [A (w2 rows) 16K][B (intermediate rows) bm*128][SFA 512][SFB 512]
+  const int off_b = kTile * kRowBytes;
+  const int off_sf = off_b + p.bm * kRowBytes;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_a = policy_evict_last();
+    const int MT2 = p.K / kTile, KT2 = p.I / 128;
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int b = u / p.n_ht, ht = u - (u / p.n_ht) * p.n_ht;
+      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      if (bi.nend == 0) continue;
+      const int w2_row = bi.e * p.K + ht * kTile;
+      const uint32_t tx = kTile * kRowBytes + bi.n16 * kRowBytes + (kFp8 ? 2 * kSfTileBytes : 0);
+      for (int kc = 0; kc < p.n_kc; ++kc) {
+        if (lane == 0) {
+          ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
+          if (ok) {
+            uint8_t* st = stage_ptr(s);
+            mbar_arrive_expect_tx(&full[s], tx);
+            tma_load_2d(st, &tm_w2, &full[s], kc * kKC, w2_row, pol_w);
+            for (int i = 0; i < bi.n16 / 16; ++i)
+              tma_load_2d(st + off_b + i * 16 * kRowBytes, &tm_act, &full[s], kc * kKC, b * p.bm + 16 * i, pol_a);
+            if (kFp8) {
+              const uint8_t* sfa = p.w2_sf + ((static_cast<int64_t>(bi.e) * MT2 + ht) * KT2 + kc) * kSfTileBytes;
+              const uint8_t* sfb = p.act_sf + (static_cast<int64_t>(b) * KT2 + kc) * kSfTileBytes;
+              bulk_load(st + off_sf, sfa, kSfTileBytes, &full[s]);
+              bulk_load(st + off_sf + kSfTileBytes, sfb, kSfTileBytes, &full[s]);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (++s == S) { s = 0; ph ^= 1u; }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    int s = 0;
+    uint32_t ph = 0;
+    int acc_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int b = u / p.n_ht;
+      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      if (bi.nend == 0) continue;
+      const int buf = acc_it % kNumAcc;
+      const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
+      if (lane == 0) ok = mbar_wait(&acc_empty[buf], acc_ph ^ 1u, abort_flag, p.status);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t d = tbase + static_cast<uint32_t>(buf) * 128u;
+      for (int kc = 0; kc < p.n_kc; ++kc) {
+        if (lane == 0) {
+          ok = mbar_wait(&full[s], ph, abort_flag, p.status);
+          if (ok) {
+            tc_fence_after();
+            uint8_t* st = stage_ptr(s);
+            const uint64_t ad = sdesc_sw128(smem_u32(st));
+            const uint64_t bd = sdesc_sw128(smem_u32(st + off_b));
+            if (kFp8) {
+              tc_cp_32x128b_x4(tbase + kP2SfCol + 0, sdesc_sf(smem_u32(st + off_sf)));
+              tc_cp_32x128b_x4(tbase + kP2SfCol + 4, sdesc_sf(smem_u32(st + off_sf + kSfTileBytes)));
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t acc = (kc | kk) != 0;
+              const uint64_t step = static_cast<uint64_t>(2 * kk);
+              if (kFp8) {
+                const uint32_t sfid = static_cast<uint32_t>(kk) << 30;
+                mma_mxf8(d, ad + step, bd + step, idesc_mxf8(kTile, bi.n16, kk, kk), (tbase + kP2SfCol) | sfid,
+                         (tbase + kP2SfCol + 4) | sfid, acc);
+              } else {
+                mma_f16(d, ad + step, bd + step, idesc_bf16(kTile, bi.n16), acc);
+              }
+            }
+            tc_commit(&empty[s]);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (++s == S) { s = 0; ph ^= 1u; }
+      }
+      if (ok && lane == 0) tc_commit(&acc_full[buf]);
+      ++acc_it;
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;
+    int acc_it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+      const int b = u / p.n_ht, ht = u - (u / p.n_ht) * p.n_ht;
+      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      if (bi.nend == 0) continue;
+      const int buf = acc_it % kNumAcc;
+      const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
+      ok = mbar_wait(&acc_full[buf], acc_ph, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 128u;
+      const int hcol = ht * kTile + 32 * q + lane;
+      const int64_t row0 = static_cast<int64_t>(b) * p.bm;
+      for (int c0 = 0; c0 < bi.nend; c0 += 16) {
+        uint32_t yr[16];
+        tmem_ld16(tacc + c0, yr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = c0 + i;
+          if (row_valid(bi, c)) {
+            const int route = __ldg(p.sorted_ids + row0 + c);
+            const float w = __ldg(p.topk_w + route);
+            p.yw[static_cast<int64_t>(route) * p.K + hcol] = w * __uint_as_float(yr[i]);
+            if (ht == 0 && q == 0 && lane == 0) p.flags[route] = 1;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      ++acc_it;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) drain_after_abort();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ========================================================================
+// combine: out[t] = bf16( sum_j yw[t*top_k + j] ), routes in order
+// ========================================================================
+__global__ void moe_combine_kernel(const float* __restrict__ yw, const int32_t* __restrict__ flags,
+                                   __nv_bfloat16* __restrict__ out, int T, int K, int top_k) {
+  const int kv = K / 8;
+  const int64_t n = static_cast<int64_t>(T) * kv;
+  for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = v / kv;
+    const int h = static_cast<int>(v - t * kv) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < top_k; ++j) {
+      const int64_t r = t * top_k + j;
+      if (__ldg(flags + r)) {
+        const float4* src = reinterpret_cast<const float4*>(yw + r * K + h);
+        const float4 a = __ldg(src), bb = __ldg(src + 1);
+        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+        acc[4] += bb.x; acc[5] += bb.y; acc[6] += bb.z; acc[7] += bb.w;
+      }
+    }
+    __nv_bfloat162 o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    *reinterpret_cast<uint4*>(out + t * K + h) = *reinterpret_cast<const uint4*>(o);
+  }
+}
+
+// ========================================================================
+// host side
+// ========================================================================
+struct WsLayout {
+  int64_t act, act_sf, yw, flags, total;
+  int64_t cap_rows;
+};
+
+static int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+static WsLayout ws_layout(bool fp8, int T, int K, int N, int E, int top_k, int bm) {
+  WsLayout w{};
+  const int64_t R = static_cast<int64_t>(T) * top_k;
+  const int64_t cap = R + static_cast<int64_t>(E) * (bm - 1);
+  w.cap_rows = round_up(cap, bm);
+  const int64_t I = N / 2;
+  int64_t off = 0;
+  w.act = off;
+  off = round_up(off + w.cap_rows * I * (fp8 ? 1 : 2), 1024);
+  w.act_sf = off;
+  if (fp8) off = round_up(off + (w.cap_rows / bm) * (I / 128) * kSfTileBytes, 1024);
+  w.yw = off;
+  off = round_up(off + R * K * 4, 1024);
+  w.flags = off;
+  off = round_up(off + R * 4, 256);
+  w.total = off;
+  return w;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D row-major [rows x cols] tensor, box [box_rows x 128 bytes], 128-byte swizzle.
+static int make_tmap(CUtensorMap* m, const void* base, bool fp8, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  const int esize = fp8 ? 1 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * esize)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kRowBytes / esize), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return MOE_OK;
+}
+
+static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+template <typename K>
+static int set_smem_attr(K kernel, int bytes, bool* done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice");
+  if (dev < kMaxDevices && done[dev]) return MOE_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
+    return cuda_fail("cudaFuncSetAttribute");
+  (void)bytes;
+  if (dev < kMaxDevices) done[dev] = true;
+  return MOE_OK;
+}
+
+struct FusedArgs {
+  bool fp8;
+  const void* x;
+  const uint8_t* x_sf;
+  const void* w1;
+  const uint8_t* w1_sf;
+  const void* w2;
+  const uint8_t* w2_sf;
+  const int32_t* sorted_ids;
+  const int32_t* expert_ids;
+  const int32_t* ntpp;
+  const float* topk_w;
+  void* out;
+  int T, K, N, E, top_k, bm;
+  int64_t capacity;
+  void* ws;
+  int64_t ws_bytes;
+  const moe_tuning* tune;
+  cudaStream_t stream;
+};
+
+static int p1_stage_bytes(bool fp8, int bm) {
+  return static_cast<int>(round_up(2 * kTile * kRowBytes + bm * kRowBytes + (fp8 ? 3 * kSfTileBytes : 0), 1024));
+}
+static int p2_stage_bytes(bool fp8, int bm) {
+  return static_cast<int>(round_up(kTile * kRowBytes + bm * kRowBytes + (fp8 ? 2 * kSfTileBytes : 0), 1024));
+}
+constexpr int kP1Ctrl = 64 * 16 + 16 + kP1GatherWarps * 128 * 4;  // barriers, tmem base, flags, token tables
+constexpr int kP2Ctrl = 64 * 16 + 16;
+
+static int pick_stages(int stage_bytes, int ctrl, int requested, int max_stages) {
+  int s = (kSmemLimit - 1024 - ctrl) / stage_bytes;
+  if (s > max_stages) s = max_stages;
+  if (requested > 0 && requested < s) s = requested;
+  return s;
+}
+
+static int run_fused(const FusedArgs& a) {
+  const char* nm = a.fp8 ? "fused_moe_mxfp8" : "fused_moe_bf16";
+  if (a.T < 0 || a.K <= 0 || a.N <= 0 || a.E < 1 || a.top_k < 1)
+    return fail(MOE_ERR_INVALID_ARG, "%s: need T >= 0, K > 0, N > 0, E >= 1, top_k >= 1", nm);
+  if (!valid_block_m(a.bm)) return fail(MOE_ERR_UNSUPPORTED, "%s: block_m must be 16, 32, 64 or 128", nm);
+  if (a.fp8) {
+    if (a.K % 256 != 0 || a.N % 256 != 0)
+      return fail(MOE_ERR_UNSUPPORTED, "%s: K and N must be multiples of 256 (K=%d N=%d)", nm, a.K, a.N);
+  } else {
+    if (a.K % 128 != 0 || a.N % 16 != 0)
+      return fail(MOE_ERR_UNSUPPORTED, "%s: K %% 128 == 0 and N %% 16 == 0 required (K=%d N=%d)", nm, a.K, a.N);
+  }
+  const int64_t need_cap = moe_align_capacity(a.T, a.top_k, a.E, a.bm);
+  if (need_cap >= (int64_t(1) << 31)) return fail(MOE_ERR_UNSUPPORTED, "%s: T*top_k + E*(block_m-1) >= 2^31", nm);
+  if (a.capacity < need_cap)
+    return fail(MOE_ERR_INVALID_ARG, "%s: capacity %lld < required %lld", nm, (long long)a.capacity,
+                (long long)need_cap);
+  if (static_cast<int64_t>(a.E) * a.N >= (int64_t(1) << 31) || static_cast<int64_t>(a.E) * a.K >= (int64_t(1) << 31))
+    return fail(MOE_ERR_UNSUPPORTED, "%s: E*N and E*K must be < 2^31", nm);
+  if (a.T == 0) return MOE_OK;
+  if (!a.x || !a.w1 || !a.w2 || !a.sorted_ids || !a.expert_ids || !a.ntpp || !a.topk_w || !a.out || !a.ws)
+    return fail(MOE_ERR_INVALID_ARG, "%s: null pointer", nm);
+  if (a.fp8 && (!a.x_sf || !a.w1_sf || !a.w2_sf)) return fail(MOE_ERR_INVALID_ARG, "%s: null scale pointer", nm);
+  if (!aligned(a.x, 16) || !aligned(a.w1, 16) || !aligned(a.w2, 16) || !aligned(a.out, 16) ||
+      !aligned(a.ws, 256) || (a.fp8 && (!aligned(a.x_sf, 16) || !aligned(a.w1_sf, 16) || !aligned(a.w2_sf, 16))) ||
+      !aligned(a.sorted_ids, 4) || !aligned(a.expert_ids, 4) || !aligned(a.ntpp, 4) || !aligned(a.topk_w, 4))
+    return fail(MOE_ERR_ALIGNMENT, "%s: tensors must be 16-byte aligned and the workspace 256-byte aligned", nm);
+  const WsLayout L = ws_layout(a.fp8, a.T, a.K, a.N, a.E, a.top_k, a.bm);
+  if (a.ws_bytes < L.total)
+    return fail(MOE_ERR_WORKSPACE, "%s: workspace %lld bytes < required %lld", nm, (long long)a.ws_bytes,
+                (long long)L.total);
+
+  const int I = a.N / 2;
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  static int* status_ptr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice");
+  if (dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "%s: device index %d too large", nm, dev);
+  if (!status_ptr[dev]) {
+    void* sp = nullptr;
+    if (cudaGetSymbolAddress(&sp, g_moe_status) != cudaSuccess) return cuda_fail("cudaGetSymbolAddress");
+    status_ptr[dev] = static_cast<int*>(sp);
+  }
+
+  CUtensorMap tm_w1, tm_w2, tm_act;
+  int rc;
+  if ((rc = make_tmap(&tm_w1, a.w1, a.fp8, static_cast<int64_t>(a.E) * a.N, a.K, kTile)) != MOE_OK) return rc;
+  if ((rc = make_tmap(&tm_w2, a.w2, a.fp8, static_cast<int64_t>(a.E) * a.K, I, kTile)) != MOE_OK) return rc;
+  if ((rc = make_tmap(&tm_act, ws + L.act, a.fp8, L.cap_rows, I, 16)) != MOE_OK) return rc;
+
+  const int nsm = sm_count();
+  if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(SM count)");
+  const int req_stages = a.tune ? a.tune->stages : 0;
+  const int req_ctas = a.tune ? a.tune->num_ctas : 0;
+  // Blocks a kernel may visit: never past the caller's sorted_token_ids /
+  // expert_ids arrays, even if num_tokens_post_padded were out of range.
+  const int max_blocks = static_cast<int>(std::min<int64_t>(L.cap_rows, a.capacity) / a.bm);
+
+  P1Params p1{};
+  p1.x = static_cast<const uint8_t*>(a.x);
+  p1.x_sf = a.x_sf;
+  p1.w1_sf = a.w1_sf;
+  p1.sorted_ids = a.sorted_ids;
+  p1.expert_ids = a.expert_ids;
+  p1.ntpp = a.ntpp;
+  p1.act = ws + L.act;
+  p1.act_sf = ws + L.act_sf;
+  p1.flags = reinterpret_cast<int32_t*>(ws + L.flags);
+  p1.status = status_ptr[dev];
+  p1.K = a.K; p1.N = a.N; p1.I = I; p1.E = a.E; p1.top_k = a.top_k; p1.bm = a.bm;
+  p1.R = a.T * a.top_k;
+  p1.max_blocks = max_blocks;
+  p1.n_jt = (I + kTile - 1) / kTile;
+  p1.stage_bytes = p1_stage_bytes(a.fp8, a.bm);
+  p1.stages = pick_stages(p1.stage_bytes, kP1Ctrl, req_stages, 8);
+
+  P2Params p2{};
+  p2.w2_sf = a.w2_sf;
+  p2.act_sf = ws + L.act_sf;
+  p2.sorted_ids = a.sorted_ids;
+  p2.expert_ids = a.expert_ids;
+  p2.ntpp = a.ntpp;
+  p2.topk_w = a.topk_w;
+  p2.yw = reinterpret_cast<float*>(ws + L.yw);
+  p2.flags = p1.flags;
+  p2.status = p1.status;
+  p2.K = a.K; p2.I = I; p2.E = a.E; p2.top_k = a.top_k; p2.bm = a.bm; p2.R = p1.R;
+  p2.max_blocks = max_blocks;
+  p2.n_ht = a.K / kTile;
+  p2.n_kc = a.fp8 ? I / 128 : (I + 63) / 64;
+  p2.stage_bytes = p2_stage_bytes(a.fp8, a.bm);
+  p2.stages = pick_stages(p2.stage_bytes, kP2Ctrl, req_stages, 8);
+  if (p1.stages < 2 || p2.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "%s: shared memory too small", nm);
+
+  const int64_t units1 = static_cast<int64_t>(max_blocks) * p1.n_jt;
+  const int64_t units2 = static_cast<int64_t>(max_blocks) * p2.n_ht;
+  int ctas = req_ctas > 0 ? req_ctas : nsm;
+  const int grid1 = static_cast<int>(units1 < ctas ? units1 : ctas);
+  const int grid2 = static_cast<int>(units2 < ctas ? units2 : ctas);
+  // Each CTA allocates all 512 TMEM columns: request more than half of the
+  // shared memory so that two CTAs never share an SM.
+  const int smem1 = std::max(1024 + p1.stages * p1.stage_bytes + kP1Ctrl, kSmemLimit / 2 + 1024);
+  const int smem2 = std::max(1024 + p2.stages * p2.stage_bytes + kP2Ctrl, kSmemLimit / 2 + 1024);
+
+  void* const* ev = a.tune ? a.tune->phase_events : nullptr;
+  auto mark = [&](int i) -> int {
+    if (ev && cudaEventRecord(static_cast<cudaEvent_t>(ev[i]), a.stream) != cudaSuccess)
+      return cuda_fail("fused_moe: cudaEventRecord");
+    return MOE_OK;
+  };
+  static bool attr_done[4][kMaxDevices] = {};
+  if (a.fp8) {
+    if ((rc = set_smem_attr(moe_p1_kernel<true>, smem1, attr_done[0])) != MOE_OK) return rc;
+    if ((rc = set_smem_attr(moe_p2_kernel<true>, smem2, attr_done[1])) != MOE_OK) return rc;
+  } else {
+    if ((rc = set_smem_attr(moe_p1_kernel<false>, smem1, attr_done[2])) != MOE_OK) return rc;
+    if ((rc = set_smem_attr(moe_p2_kernel<false>, smem2, attr_done[3])) != MOE_OK) return rc;
+  }
+  if ((rc = mark(0)) != MOE_OK) return rc;
+  if (a.fp8) moe_p1_kernel<true><<<grid1, kP1Threads, smem1, a.stream>>>(tm_w1, p1);
+  else moe_p1_kernel<false><<<grid1, kP1Threads, smem1, a.stream>>>(tm_w1, p1);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return cuda_fail("fused_moe: gate/up phase launch", err);
+  if ((rc = mark(1)) != MOE_OK) return rc;
+  if (a.fp8) moe_p2_kernel<true><<<grid2, kP2Threads, smem2, a.stream>>>(tm_w2, tm_act, p2);
+  else moe_p2_kernel<false><<<grid2, kP2Threads, smem2, a.stream>>>(tm_w2, tm_act, p2);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return cuda_fail("fused_moe: down phase launch", err);
+  if ((rc = mark(2)) != MOE_OK) return rc;
+  const int64_t nvec = static_cast<int64_t>(a.T) * (a.K / 8);
+  const int64_t cblocks = (nvec + 255) / 256;
+  moe_combine_kernel<<<static_cast<int>(cblocks < 4L * nsm ? cblocks : 4L * nsm), 256, 0, a.stream>>>(
+      reinterpret_cast<const float*>(ws + L.yw), p1.flags, static_cast<__nv_bfloat16*>(a.out), a.T, a.K,
+      a.top_k);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return cuda_fail("fused_moe: combine launch", err);
+  return mark(3);
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" int64_t moe_workspace_bytes(int dtype, int T, int K, int N, int E, int top_k, int block_m) {
+  if (T < 0 || K <= 0 || N <= 0 || E < 1 || top_k < 1 || !valid_block_m(block_m)) return -1;
+  if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_MXFP8) return -1;
+  return ws_layout(dtype == MOE_DTYPE_MXFP8, T, K, N, E, top_k, block_m).total;
+}
+
+extern "C" int moe_device_status(moe_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return cuda_fail("moe_device_status: cudaStreamSynchronize");
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_moe_status, sizeof(int)) != cudaSuccess)
+    return cuda_fail("moe_device_status: read");
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_moe_status, &zero, sizeof(int)) != cudaSuccess)
+      return cuda_fail("moe_device_status: clear");
+    return fail(v, "a device-side wait timed out");
+  }
+  return MOE_OK;
+}
+
+extern "C" int fused_moe_bf16(const void* x, const void* w1, const void* w2, const int32_t* sorted_token_ids,
+                              const int32_t* expert_ids, const int32_t* num_tokens_post_padded,
+                              const float* topk_weights, void* out, int T, int K, int N, int E, int top_k,
+                              int block_m, int64_t capacity, void* workspace, int64_t workspace_bytes,
+                              const moe_tuning* tune, moe_stream_t stream) {
+  FusedArgs a{};
+  a.fp8 = false;
+  a.x = x; a.w1 = w1; a.w2 = w2;
+  a.sorted_ids = sorted_token_ids; a.expert_ids = expert_ids; a.ntpp = num_tokens_post_padded;
+  a.topk_w = topk_weights; a.out = out;
+  a.T = T; a.K = K; a.N = N; a.E = E; a.top_k = top_k; a.bm = block_m; a.capacity = capacity;
+  a.ws = workspace; a.ws_bytes = workspace_bytes; a.tune = tune;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  return run_fused(a);
+}
+
+extern "C" int fused_moe_mxfp8(const uint8_t* x_e4m3, const uint8_t* x_scales, const uint8_t* w1_e4m3,
+                               const uint8_t* w1_scales_blocked, const uint8_t* w2_e4m3,
+                               const uint8_t* w2_scales_blocked, const int32_t* sorted_token_ids,
+                               const int32_t* expert_ids, const int32_t* num_tokens_post_padded,
+                               const float* topk_weights, void* out, int T, int K, int N, int E, int top_k,
+                               int block_m, int64_t capacity, void* workspace, int64_t workspace_bytes,
+                               const moe_tuning* tune, moe_stream_t stream) {
+  FusedArgs a{};
+  a.fp8 = true;
+  a.x = x_e4m3; a.x_sf = x_scales; a.w1 = w1_e4m3; a.w1_sf = w1_scales_blocked;
+  a.w2 = w2_e4m3; a.w2_sf = w2_scales_blocked;
+  a.sorted_ids = sorted_token_ids; a.expert_ids = expert_ids; a.ntpp = num_tokens_post_padded;
+  a.topk_w = topk_weights; a.out = out;
+  a.T = T; a.K = K; a.N = N; a.E = E; a.top_k = top_k; a.bm = block_m; a.capacity = capacity;
+  a.ws = workspace; a.ws_bytes = workspace_bytes; a.tune = tune;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  return run_fused(a);
+}

@@ -1,0 +1,144 @@
+"""Fused MoE forward on the GPU (planner + fused kernels, through the C ABI)
+against the oracle on the same seeded inputs.
+
+bf16 path: max|gpu - oracle| <= 2e-2 * rms(oracle out).
+mxfp8 path (the oracle emulates the on-chip requant): cosine >= 0.999 and
+max|gpu - oracle| <= 6e-2 * rms(oracle out).  "oracle out" is the oracle's
+result before its final rounding to bf16 (see tests/helpers.py).
+Small cases run the whole oracle; they span several 128-row blocks, several
+intermediate tiles and a ragged tail.  The named workloads at full size are
+checked on a seeded token sample that always includes tokens of the most-
+and least-loaded experts (tokens are independent, so their rows are exact
+sub-results).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as W
+from tests.helpers import assert_bf16_parity, assert_mxfp8_parity, out_bits, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_forward(sh: W.Shape, inp: dict, block_m: int | None = None, tune=None, repeat: int = 1):
+    """Uploads the inputs, runs moe_align + fused_moe_*; returns host bf16 bits (T, K) per repeat."""
+    import torch
+    import mixture_experts_ffn_planner_b200 as moe
+
+    bm = block_m or sh.block_m
+    ids = to_dev(inp["topk_ids"])
+    tw = to_dev(inp["topk_weights"])
+    sorted_ids, expert_ids, ntpp = moe.moe_align(ids, sh.E, bm)
+    outs = []
+    if sh.dtype == "bf16":
+        x, w1, w2 = (to_dev(inp[n], torch.bfloat16) for n in ("x", "w1", "w2"))
+        for _ in range(repeat):
+            out = torch.full((sh.T, sh.K), float("nan"), dtype=torch.bfloat16, device="cuda")
+            moe.fused_moe_bf16(x, w1, w2, sorted_ids, expert_ids, ntpp, tw, out, bm, tune=tune)
+            outs.append(out)
+    else:
+        x, xs, w1, w2 = (to_dev(inp[n]) for n in ("x", "x_scales", "w1", "w2"))
+        s1 = moe.pack_scales_blocked(to_dev(inp["w1_scales"]))
+        s2 = moe.pack_scales_blocked(to_dev(inp["w2_scales"]))
+        for _ in range(repeat):
+            out = torch.full((sh.T, sh.K), float("nan"), dtype=torch.bfloat16, device="cuda")
+            moe.fused_moe_mxfp8(x, xs, w1, s1, w2, s2, sorted_ids, expert_ids, ntpp, tw, out, bm, tune=tune)
+            outs.append(out)
+    moe.moe_device_status()
+    res = [out_bits(o) for o in outs]
+    return res if repeat > 1 else res[0]
+
+
+def oracle_forward(sh: W.Shape, inp: dict, tokens=None):
+    """The oracle's out before its final bf16 rounding (float64, (T, K))."""
+    if sh.dtype == "bf16":
+        return oracle.fused_moe_bf16(inp["x"], inp["w1"], inp["w2"], inp["topk_ids"], inp["topk_weights"],
+                                     tokens=tokens, unrounded=True)[1]
+    return oracle.fused_moe_mxfp8(inp["x"], inp["x_scales"], inp["w1"], inp["w1_scales"], inp["w2"],
+                                  inp["w2_scales"], inp["topk_ids"], inp["topk_weights"], tokens=tokens,
+                                  unrounded=True)[1]
+
+
+def check(sh, got, ref, what):
+    if sh.dtype == "bf16":
+        return assert_bf16_parity(got, ref, what)
+    return assert_mxfp8_parity(got, ref, what)
+
+
+def small(dtype, T, K, N, E, top_k, block_m, zipf=None):
+    return W.Shape(name="S", dtype=dtype, T=T, K=K, N=N, E=E, top_k=top_k, block_m=block_m, zipf_s=zipf)
+
+
+SMALL_BF16 = [
+    small("bf16", 200, 256, 512, 8, 2, 128),      # 2 intermediate tiles, ragged blocks
+    small("bf16", 200, 256, 512, 8, 2, 64),
+    small("bf16", 77, 128, 320, 5, 3, 32),        # I = 160: partial intermediate tile
+    small("bf16", 50, 384, 80, 6, 2, 16),         # I = 40: partial 64-wide K chunk in the down GEMM
+    small("bf16", 300, 256, 256, 16, 4, 128, 1.2),  # skewed routing, empty experts
+    small("bf16", 1, 128, 256, 4, 1, 128),
+]
+SMALL_MXFP8 = [
+    small("mxfp8", 200, 256, 512, 8, 2, 128),
+    small("mxfp8", 200, 512, 256, 8, 2, 64),
+    small("mxfp8", 90, 256, 768, 6, 3, 32),       # I = 384: 3 intermediate tiles
+    small("mxfp8", 300, 256, 256, 16, 4, 128, 1.2),
+]
+
+
+@pytest.mark.parametrize("sh", SMALL_BF16 + SMALL_MXFP8, ids=lambda s: f"{s.dtype}-T{s.T}-K{s.K}-N{s.N}-E{s.E}-"
+                         f"k{s.top_k}-bm{s.block_m}")
+def test_small_full_oracle(sh):
+    inp = W.inputs(sh, seed=11)
+    got = gpu_forward(sh, inp)
+    ref = oracle_forward(sh, inp)
+    check(sh, got, ref, "small")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "mxfp8"])
+def test_deterministic(dtype):
+    sh = small(dtype, 300, 256, 512, 8, 3, 128)
+    a, b = gpu_forward(sh, W.inputs(sh, seed=3), repeat=2)
+    np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "mxfp8"])
+def test_invalid_routes_contribute_nothing(dtype):
+    """Routes whose expert id is outside [0, E) get no slot and add nothing."""
+    sh = small(dtype, 64, 256, 256, 4, 2, 128)
+    inp = W.inputs(sh, seed=4)
+    inp["topk_ids"] = inp["topk_ids"].copy()
+    inp["topk_ids"][::3, 1] = -1
+    inp["topk_ids"][5, :] = 9
+    got = gpu_forward(sh, inp)
+    ref = oracle_forward(sh, inp)
+    check(sh, got, ref, "invalid ids")
+    assert not got[5].any() or np.all((got[5] & 0x7FFF) == 0)
+
+
+@pytest.mark.parametrize("stages", [2, 3])
+def test_tuning_stages(stages):
+    import mixture_experts_ffn_planner_b200 as moe
+
+    sh = small("bf16", 150, 512, 512, 8, 2, 128)
+    inp = W.inputs(sh, seed=8)
+    got = gpu_forward(sh, inp, tune=moe.Tuning(stages=stages, num_ctas=7))
+    check(sh, got, oracle_forward(sh, inp), f"stages={stages}")
+
+
+def test_c1_full():
+    """bf16, T=64, K=1024, N=1024, E=8, top-2, block_m=64: whole oracle."""
+    sh = W.shape("C1", 64)
+    inp = W.inputs(sh)
+    check(sh, gpu_forward(sh, inp), oracle_forward(sh, inp), "C1")
+
+
+@pytest.mark.parametrize("T", [1, 8, 64, 512, 8192])
+def test_c5_sampled(T):
+    """bf16 narrow intermediate with Zipf-skewed routing (empty experts)."""
+    sh = W.shape("C5", T)
+    inp = W.inputs(sh)
+    toks = W.sample_tokens(sh, inp["topk_ids"], 48)
+    got = gpu_forward(sh, inp)
+    ref = oracle_forward(sh, inp, tokens=toks)
+    check(sh, got[toks], ref[toks], f"C5 T={T}")
