@@ -50,17 +50,20 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--workload", default="C2", choices=W.workload_names())
     ap.add_argument("--tokens", type=int, default=256)
+    ap.add_argument("--experts", type=int, default=0, help="override the workload's expert count (profiling)")
     ap.add_argument("--seed", type=int, default=W.DEFAULT_SEED)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--stages", type=int, default=0)
     ap.add_argument("--ctas", type=int, default=0)
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="flush L2 between steps (automatic when the touched weights are < 4x L2)")
     return ap.parse_args(argv)
 
 
@@ -205,7 +208,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    sh = W.shape(args.workload, args.tokens)
+    sh = W.shape(args.workload, args.tokens, **({"E": args.experts} if args.experts else {}))
     inp = W.inputs(sh, seed=args.seed)
     thr = os.cpu_count() or 1
     # calibrate: tokens per step such that all steps fit in ~2 minutes
@@ -238,11 +241,195 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+class Problem:
+    """Device-resident inputs of one workload and one step of the hot path."""
+
+    def __init__(self, sh: W.Shape, inp: dict, dev, stages: int = 0, ctas: int = 0):
+        import torch
+
+        import mixture_experts_ffn_planner_b200 as moe
+
+        self.sh, self.inp, self.dev, self.moe = sh, inp, dev, moe
+
+        def up(a, dtype=None):
+            t = torch.from_numpy(np.ascontiguousarray(a))
+            return (t.view(dtype) if dtype is not None else t).to(dev)
+
+        bm = self.bm = sh.block_m
+        self.ids, self.tw = up(inp["topk_ids"]), up(inp["topk_weights"])
+        cap = moe.moe_align_capacity(sh.T, sh.top_k, sh.E, bm)
+        self.s_ids = torch.empty(cap, dtype=torch.int32, device=dev)
+        self.e_ids = torch.empty((cap + bm - 1) // bm, dtype=torch.int32, device=dev)
+        self.ntpp = torch.empty(1, dtype=torch.int32, device=dev)
+        self.out = torch.empty((sh.T, sh.K), dtype=torch.bfloat16, device=dev)
+        if sh.dtype == "bf16":
+            self.x = up(inp["x"], torch.bfloat16)
+            self.w1, self.w2 = up(inp["w1"], torch.bfloat16), up(inp["w2"], torch.bfloat16)
+            self.xs = self.s1 = self.s2 = None
+            dt = moe.DTYPE_BF16
+        else:
+            self.x, self.xs, self.w1, self.w2 = up(inp["x"]), up(inp["x_scales"]), up(inp["w1"]), up(inp["w2"])
+            self.s1 = moe.pack_scales_blocked(up(inp["w1_scales"]))
+            self.s2 = moe.pack_scales_blocked(up(inp["w2_scales"]))
+            dt = moe.DTYPE_MXFP8
+        self.ws = torch.empty(moe.moe_workspace_bytes(dt, sh.T, sh.K, sh.N, sh.E, sh.top_k, bm),
+                              dtype=torch.uint8, device=dev)
+        self.plain = moe.Tuning(stages, ctas, None)
+        self.stages, self.ctas = stages, ctas
+        self.launches_per_step = 4  # moe_align, gate/up phase, down phase, reduction
+
+    def fused(self, tune):
+        m = self.moe
+        if self.sh.dtype == "bf16":
+            m.fused_moe_bf16(self.x, self.w1, self.w2, self.s_ids, self.e_ids, self.ntpp, self.tw, self.out, self.bm,
+                             workspace=self.ws, tune=tune)
+        else:
+            m.fused_moe_mxfp8(self.x, self.xs, self.w1, self.s1, self.w2, self.s2, self.s_ids, self.e_ids, self.ntpp,
+                              self.tw, self.out, self.bm, workspace=self.ws, tune=tune)
+
+    def step(self, tune=None):
+        self.moe.moe_align(self.ids, self.sh.E, self.bm, self.s_ids, self.e_ids, self.ntpp)
+        self.fused(self.plain if tune is None else tune)
+
+
+def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barrier=None, sample_clocks=True,
+            local: int = 0):
+    """Device time of `steps` steps after `warmup`.  With flush_l2 every step is
+    bracketed by its own events and a >L2 buffer is written between steps
+    (outside the timed windows); otherwise the steps run back to back between
+    one pair of events.  The library's phase events time each kernel."""
+    import torch
+
+    moe = prob.moe
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    tunes = [moe.Tuning.with_events(e, prob.stages, prob.ctas) for e in ev]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=prob.dev) if flush_l2 else None
+    for _ in range(max(3, warmup)):
+        prob.step()
+        if flush is not None:
+            flush.fill_(1)
+    moe.moe_device_status()
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local) if sample_clocks else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)] \
+        if flush_l2 else None
+    t0.record(stream)
+    for i in range(steps):
+        if s_ev:
+            s_ev[i][0].record(stream)
+        prob.step(tunes[i])
+        if s_ev:
+            s_ev[i][1].record(stream)
+            flush.fill_(1)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    clk = clocks.stop() if clocks else None
+    moe.moe_device_status()
+    if s_ev:
+        total_ms = sum(a.elapsed_time(b) for a, b in s_ev)
+    else:
+        total_ms = t0.elapsed_time(t1)
+    return {"total_ms": total_ms, "ms_step": total_ms / steps,
+            "p1_ms": sum(e[0].elapsed_time(e[1]) for e in ev) / steps,
+            "p2_ms": sum(e[1].elapsed_time(e[2]) for e in ev) / steps,
+            "cb_ms": sum(e[2].elapsed_time(e[3]) for e in ev) / steps,
+            "clocks": clk, "launches": prob.launches_per_step * steps}
+
+
+def measure_e2e(prob: Problem, steps: int, barrier=None):
+    """Same steps through host buffers: pinned H2D of the step's inputs (x, its
+    scales, routing) and D2H of out inside the timed region."""
+    import torch
+
+    sh, inp = prob.sh, prob.inp
+    stream = torch.cuda.current_stream()
+    hx = torch.from_numpy(np.ascontiguousarray(inp["x"]))
+    hx = hx.view(torch.bfloat16) if sh.dtype == "bf16" else hx
+    host_in = [hx.pin_memory(), torch.from_numpy(inp["topk_ids"]).pin_memory(),
+               torch.from_numpy(inp["topk_weights"]).pin_memory()]
+    dev_in = [prob.x, prob.ids, prob.tw]
+    if sh.dtype == "mxfp8":
+        host_in.append(torch.from_numpy(np.ascontiguousarray(inp["x_scales"])).pin_memory())
+        dev_in.append(prob.xs)
+    host_out = torch.empty((sh.T, sh.K), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def one():
+        for h, d in zip(host_in, dev_in):
+            d.copy_(h, non_blocking=True)
+        prob.step()
+        host_out.copy_(prob.out, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1), h2d, d2h
+
+
+def roofline_of_p1(sh: W.Shape, cm: dict, p1_ms: float, peaks: dict, peak_src: str):
+    p1_s = p1_ms * 1e-3
+    tag = f"{sh.name}_T{sh.T}"
+    name = "moe_p1_kernel (gather + gate/up GEMM + SwiGLU)"
+    if cm["p1_flops"] / cm["p_tc"] <= cm["p1_bytes"] / cm["bw"]:
+        gbs = cm["p1_bytes"] / p1_s / 1e9
+        return {"kernel": name, "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"], "traffic": kernel_traffic("moe_p1_kernel", tag),
+                "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": cm["p1_bytes"],
+                "us_per_launch": p1_ms * 1e3}
+    pk = peaks["bf16_tflops"] * (1.0 if sh.dtype == "bf16" else 2.0)
+    tf = cm["p1_flops"] / p1_s / 1e12
+    return {"kernel": name, "bound": "tensor", "achieved": tf, "peak": pk, "unit": "TFLOP/s", "frac": tf / pk,
+            "traffic": kernel_traffic("moe_p1_kernel", tag),
+            "peak_source": f"{peak_src} bf16_tflops" + ("" if sh.dtype == "bf16" else " x 2 (fp8:bf16 nominal)"),
+            "algorithmic_flops_per_launch": cm["p1_flops"], "us_per_launch": p1_ms * 1e3}
+
+
+def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
+    ms_step = m["ms_step"]
+    l2 = ("L2 flushed between steps (512 MB write outside the per-step events)" if flush_l2 else
+          f"inputs larger than L2 (touched expert weights {cm['bytes_w'] / 1e9:.2f} GB per step)")
+    return {
+        "metric": METRIC, "value": world * cm["flops"] / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype,
+        "data": "synthetic (seeded workloads generator, random weights)",
+        "config": {"workload": f"{sh.name}: {sh.dtype} MoE FFN K={sh.K} N={sh.N} (intermediate {sh.I}) "
+                               f"E={sh.E} top_k={sh.top_k} T={sh.T} block_m={sh.block_m}",
+                   "tokens_per_gpu": sh.T, "parallelism": f"replicas x{world}", "l2": l2},
+        "us_per_call": ms_step * 1e3,
+        "weight_GBps": cm["bytes_w"] / (ms_step * 1e-3) / 1e9,
+        "path_roofline": {"bound": cm["bound"], "t_roof_us": cm["t_roof"] * 1e6,
+                          "frac": cm["t_roof"] / (ms_step * 1e-3), "touched_experts": cm["touched"],
+                          "routed_gflop": cm["flops"] / 1e9, "touched_weight_gb": cm["bytes_w"] / 1e9,
+                          "peaks": peak_src},
+        "phase_us": {"gate_up": m["p1_ms"] * 1e3, "down": m["p2_ms"] * 1e3, "reduce": m["cb_ms"] * 1e3},
+        "roofline": roofline_of_p1(sh, cm, m["p1_ms"], peaks, peak_src),
+        "gpu_launches": m["launches"],
+        "clocks": m["clocks"],
+    }
+
+
 def run_b200(args):
     import torch
     import torch.distributed as dist
-
-    import mixture_experts_ffn_planner_b200 as moe
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -253,167 +440,38 @@ def run_b200(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
+    barrier = dist.barrier if world > 1 else None
     dev = torch.device("cuda", local)
     peaks, peak_src = load_peaks()
 
-    sh = W.shape(args.workload, args.tokens)
+    sh = W.shape(args.workload, args.tokens, **({"E": args.experts} if args.experts else {}))
     inp = W.inputs(sh, seed=args.seed + rank)  # every replica gets its own batch
     cm = cost_model(sh, inp["topk_ids"], peaks)
+    prob = Problem(sh, inp, dev, args.stages, args.ctas)
+    flush = args.flush_l2 or cm["bytes_w"] < 4 * 126e6
+    m = measure(prob, args.steps, args.warmup, flush_l2=flush, barrier=barrier, local=local)
 
-    def up(a, dtype=None):
-        t = torch.from_numpy(np.ascontiguousarray(a))
-        return (t.view(dtype) if dtype is not None else t).to(dev)
-
-    ids, tw = up(inp["topk_ids"]), up(inp["topk_weights"])
-    bm = sh.block_m
-    cap = moe.moe_align_capacity(sh.T, sh.top_k, sh.E, bm)
-    s_ids = torch.empty(cap, dtype=torch.int32, device=dev)
-    e_ids = torch.empty((cap + bm - 1) // bm, dtype=torch.int32, device=dev)
-    ntpp = torch.empty(1, dtype=torch.int32, device=dev)
-    out = torch.empty((sh.T, sh.K), dtype=torch.bfloat16, device=dev)
-    if sh.dtype == "bf16":
-        x, w1, w2 = up(inp["x"], torch.bfloat16), up(inp["w1"], torch.bfloat16), up(inp["w2"], torch.bfloat16)
-        ws = torch.empty(moe.moe_workspace_bytes(moe.DTYPE_BF16, sh.T, sh.K, sh.N, sh.E, sh.top_k, bm),
-                         dtype=torch.uint8, device=dev)
-
-        def fused(tune):
-            moe.fused_moe_bf16(x, w1, w2, s_ids, e_ids, ntpp, tw, out, bm, workspace=ws, tune=tune)
-    else:
-        x, xs, w1, w2 = up(inp["x"]), up(inp["x_scales"]), up(inp["w1"]), up(inp["w2"])
-        s1 = moe.pack_scales_blocked(up(inp["w1_scales"]))
-        s2 = moe.pack_scales_blocked(up(inp["w2_scales"]))
-        ws = torch.empty(moe.moe_workspace_bytes(moe.DTYPE_MXFP8, sh.T, sh.K, sh.N, sh.E, sh.top_k, bm),
-                         dtype=torch.uint8, device=dev)
-
-        def fused(tune):
-            moe.fused_moe_mxfp8(x, xs, w1, s1, w2, s2, s_ids, e_ids, ntpp, tw, out, bm, workspace=ws, tune=tune)
-
-    stream = torch.cuda.current_stream()
-    n_ev = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_ev)]
-    tunes = [moe.Tuning.with_events(e, args.stages, args.ctas) for e in ev]
-    plain = moe.Tuning(args.stages, args.ctas, None)
-
-    def step(tune):
-        moe.moe_align(ids, sh.E, bm, s_ids, e_ids, ntpp)
-        fused(tune)
-
-    for _ in range(max(3, args.warmup)):
-        step(plain)
-    moe.moe_device_status()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(args.steps):
-        step(tunes[i])
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    moe.moe_device_status()
-    ms_local = t_start.elapsed_time(t_end)
-    p1_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
-    p2_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
-    cb_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / args.steps
-    ms = ms_local
-    if world > 1:
-        t = torch.tensor([ms_local], device=dev, dtype=torch.float64)
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    ms_step = ms / args.steps
-    value = world * cm["flops"] / (ms_step * 1e-3) / 1e12
+        return float(t.item())
 
-    # ---- end to end through the public API with host buffers
-    e2e = None
+    m["ms_step"] = max_over_ranks(m["ms_step"])
+    line = result_line(sh, cm, m, world, args.steps, args.warmup, peaks, peak_src, flush)
     if not args.no_e2e:
-        hx = torch.from_numpy(np.ascontiguousarray(inp["x"]))
-        hx = hx.view(torch.bfloat16) if sh.dtype == "bf16" else hx
-        host_in = [hx.pin_memory(), torch.from_numpy(inp["topk_ids"]).pin_memory(),
-                   torch.from_numpy(inp["topk_weights"]).pin_memory()]
-        if sh.dtype == "mxfp8":
-            host_in.append(torch.from_numpy(np.ascontiguousarray(inp["x_scales"])).pin_memory())
-        dev_in = [x, ids, tw] + ([xs] if sh.dtype == "mxfp8" else [])
-        host_out = torch.empty((sh.T, sh.K), dtype=torch.bfloat16).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host_in)
-        d2h = host_out.numel() * host_out.element_size()
-        for _ in range(3):
-            for h, d in zip(host_in, dev_in):
-                d.copy_(h, non_blocking=True)
-            step(plain)
-            host_out.copy_(out, non_blocking=True)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            for h, d in zip(host_in, dev_in):
-                d.copy_(h, non_blocking=True)
-            step(plain)
-            host_out.copy_(out, non_blocking=True)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * cm["flops"] / (ems / args.steps * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "us_per_call": 1e3 * ems / args.steps}
-
-    # ---- dominant kernel (gate/up phase) against its roofline
-    p1_s = p1_ms * 1e-3
-    p1_tflops = cm["p1_flops"] / p1_s / 1e12
-    p1_gbs = cm["p1_bytes"] / p1_s / 1e9
-    p1_bound = "tensor" if cm["p1_flops"] / cm["p_tc"] > cm["p1_bytes"] / cm["bw"] else "hbm"
-    tag = f"{sh.name}_T{sh.T}"
-    if p1_bound == "hbm":
-        roof = {"kernel": "moe_p1_kernel (gather + gate/up GEMM + SwiGLU)", "bound": "hbm", "achieved": p1_gbs,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": p1_gbs / peaks["hbm_gbs"],
-                "traffic": kernel_traffic("moe_p1_kernel", tag), "peak_source": f"{peak_src} hbm_gbs",
-                "algorithmic_bytes_per_launch": cm["p1_bytes"], "us_per_launch": p1_ms * 1e3}
-    else:
-        pk = peaks["bf16_tflops"] * (1.0 if sh.dtype == "bf16" else 2.0)
-        roof = {"kernel": "moe_p1_kernel (gather + gate/up GEMM + SwiGLU)", "bound": "tensor",
-                "achieved": p1_tflops, "peak": pk, "unit": "TFLOP/s", "frac": p1_tflops / pk,
-                "traffic": kernel_traffic("moe_p1_kernel", tag),
-                "peak_source": f"{peak_src} bf16_tflops" + ("" if sh.dtype == "bf16" else " x 2 (fp8:bf16 nominal)"),
-                "algorithmic_flops_per_launch": cm["p1_flops"], "us_per_launch": p1_ms * 1e3}
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": sh.dtype, "data": "synthetic (seeded workloads generator, random weights)",
-        "config": {"workload": f"{sh.name}: {sh.dtype} MoE FFN K={sh.K} N={sh.N} (intermediate {sh.I}) "
-                               f"E={sh.E} top_k={sh.top_k} T={sh.T} block_m={bm}",
-                   "tokens_per_gpu": sh.T, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2 (touched expert weights {cm['bytes_w'] / 1e9:.2f} GB per step)"},
-        "us_per_call": ms_step * 1e3,
-        "weight_GBps": cm["bytes_w"] / (ms_step * 1e-3) / 1e9,
-        "path_roofline": {"bound": cm["bound"], "t_roof_us": cm["t_roof"] * 1e6, "frac": cm["t_roof"] / (ms_step * 1e-3),
-                          "touched_experts": cm["touched"], "routed_gflop": cm["flops"] / 1e9,
-                          "touched_weight_gb": cm["bytes_w"] / 1e9, "peaks": peak_src},
-        "phase_us": {"gate_up": p1_ms * 1e3, "down": p2_ms * 1e3, "reduce": cb_ms * 1e3},
-        "roofline": roof,
-        "e2e": e2e,
-        "gpu_launches": 4 * args.steps,
-        "clocks": clk,
-    }
+        ems, h2d, d2h = measure_e2e(prob, args.steps, barrier)
+        ems = max_over_ranks(ems)
+        line["e2e"] = {"value": world * cm["flops"] / (ems / args.steps * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                       "us_per_call": 1e3 * ems / args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, thr, desc, spent = oracle_sample_rate(sh, inp, args.cpu_seconds, args.seed)
         line["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                                 "sample": desc, "seconds": spent}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del tunes
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

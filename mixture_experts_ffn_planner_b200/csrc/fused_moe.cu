@@ -8,27 +8,30 @@
 // requantisation of a to e4m3 + e8m0 per 32 on chip, the down GEMM
 // Y = w2[e] a, and the top-k weighted reduction out[t] = sum_j w[t,j] Y.
 //
-// How (sm_100a):
+// How (sm_100a), token-major tiles:
 //   phase 1  persistent kernel, one CTA per SM.  A work unit is (planner block
-//            b, intermediate tile j of 128 columns).  The expert's weights are
-//            the 128-row A operand of tcgen05.mma (gate rows and up rows, one
-//            MMA each), the block's gathered token rows are the B operand, so
-//            the MMA's N is the number of routed rows rounded up to 16 and the
-//            accumulators live in TMEM as [weight row (lane)] x [token
-//            (column)].  Gate row i and up row i land in the same TMEM lane,
-//            so one thread computes silu(g)*u for its intermediate column and
-//            (mxfp8) takes the 32-wide amax with one warp redux.  The
-//            intermediate is written once to an L2-resident workspace.
+//            b, intermediate tile j of 128 columns).  The block's routed token
+//            rows (gathered by cp.async into the 128-byte-swizzled layout) are
+//            the M = 128 operand of tcgen05.mma; the expert's 128 gate rows and
+//            128 up rows, streamed by TMA, form one N = 256 operand, so one MMA
+//            per 32-byte K slice fills a TMEM accumulator laid out as [token
+//            (lane)] x [gate 0..127 | up 0..127].  Each epilogue thread owns one
+//            token row: SwiGLU, the 32-wide amax, the e8m0 scale and the e4m3
+//            codes all stay in its registers, and the intermediate row segment
+//            is written with 16-byte stores into an L2-resident workspace.
 //            Warp roles: 0 TMA producer (weight tiles, weight scale tiles),
-//            1 MMA issuer, 2-5 token gather (cp.async, 128-byte swizzle, token
-//            scales), 6-9 epilogue.
-//   phase 2  persistent kernel, unit = (block b, 128 output features).  A =
-//            w2[e] rows, B = the block's intermediate rows (TMA), D in TMEM;
-//            the epilogue scales by the routing weight and writes one fp32 row
-//            per route.
+//            1 MMA issuer, 2-3 token gather (cp.async of the routed rows and,
+//            on mxfp8, their scales; completion is tracked by the stage's
+//            mbarrier, so the gather warps never wait on their own copies),
+//            4-11 epilogue (two warps per TMEM lane quadrant, one per column
+//            half).
+//   phase 2  persistent kernel, unit = (block b, 256 output features).  A =
+//            the block's intermediate rows (TMA), B = 256 rows of w2[e] (TMA),
+//            D in TMEM; each epilogue thread scales its row by the routing
+//            weight and writes one fp32 row segment per route.
 //   combine  out[t] = bf16(sum over the token's routes, in route order), a
 //            deterministic HBM-bound pass.
-// The weight tile of a unit is streamed once through a multi-stage shared
+// The weight tiles are streamed once per unit through a multi-stage shared
 // memory ring by TMA; the weights are the dominant HBM traffic.
 #include <algorithm>
 #include <mutex>
@@ -40,18 +43,28 @@ namespace moe {
 
 __device__ int g_moe_status = 0;
 
-constexpr int kTile = 128;        // weight rows per MMA (M) and features per unit
+constexpr int kM = 128;           // MMA M: routed rows of one planner block (rows >= block_m unused)
+constexpr int kTI = 128;          // intermediate columns per phase-1 unit (gate 128 + up 128 = MMA N 256)
+constexpr int kTH = 256;          // output features per phase-2 unit (MMA N)
 constexpr int kRowBytes = 128;    // bytes of one operand row per pipeline stage
 constexpr int kSfTileBytes = 512; // one blocked scale tile: 128 rows x 4 scales
 constexpr int kSmemLimit = 232448;  // 227 KB of dynamic shared memory per CTA
 
-// TMEM column map
-constexpr uint32_t kP1SfCol = 256;  // mxfp8 scale factors (12 columns) in phase 1
-constexpr uint32_t kP2SfCol = 256;  // mxfp8 scale factors (8 columns) in phase 2
+// TMEM column map: accumulators first; on the mxfp8 path (one accumulator)
+// the scale factors follow it.
+constexpr uint32_t kSfaCol = 256;   // 4 columns: 128 rows of A
+constexpr uint32_t kSfbCol = 260;   // 8 columns: 256 rows of B
 
-constexpr int kP1Threads = 320;  // 10 warps
-constexpr int kP1GatherWarps = 4;
-constexpr int kP2Threads = 192;  // 6 warps
+constexpr int kEpiWarps = 8;
+constexpr int kGatherWarps = 2;
+constexpr int kP1FirstEpi = 2 + kGatherWarps;
+constexpr int kP1Threads = 32 * (kP1FirstEpi + kEpiWarps);  // 12 warps
+constexpr int kP2FirstEpi = 2;
+constexpr int kP2Threads = 32 * (kP2FirstEpi + kEpiWarps);  // 10 warps
+
+// Stage layout (both phases): [A 128 rows x 128 B][B 256 rows x 128 B][SFA 512][SFB 2 x 512]
+constexpr int kOffB = kM * kRowBytes;
+constexpr int kOffSf = kOffB + 2 * 128 * kRowBytes;
 
 struct P1Params {
   const uint8_t* x;         // (T, K) bf16 or e4m3
@@ -61,11 +74,11 @@ struct P1Params {
   const int32_t* expert_ids;
   const int32_t* ntpp;
   uint8_t* act;             // (cap_rows, I) bf16 or e4m3
-  uint8_t* act_sf;          // blocked scales of act, one tile row per block (mxfp8)
+  uint8_t* act_sf;          // blocked scales of act, one tile per (block, 128 intermediate columns) (mxfp8)
   int32_t* flags;           // one per route, cleared here
   int* status;
   int K, N, I, E, top_k, bm, R;
-  int max_blocks;           // workspace rows / bm
+  int max_blocks;           // blocks a kernel may visit
   int n_jt;                 // ceil(I / 128)
   int stages, stage_bytes;
 };
@@ -82,7 +95,7 @@ struct P2Params {
   int* status;
   int K, I, E, top_k, bm, R;
   int max_blocks;
-  int n_ht;                 // K / 128
+  int n_ht;                 // ceil(K / 256)
   int n_kc;                 // K-chunks of the down GEMM
   int stages, stage_bytes;
 };
@@ -91,7 +104,7 @@ struct P2Params {
 struct BlockInfo {
   int e;            // expert of the block
   int nend;         // 1 + index of the last routed row in the block (0: none)
-  int n16;          // MMA N: nend rounded up to 16
+  int n16;          // nend rounded up to 16
   uint32_t vm[4];   // routed-row mask, rows 32q .. 32q+31
 };
 
@@ -139,6 +152,11 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 // ========================================================================
 // phase 1: gate/up GEMM + SwiGLU (+ mxfp8 requant) -> intermediate
 // ========================================================================
@@ -155,7 +173,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sm + 1);
-  int32_t* tok_tab = reinterpret_cast<int32_t*>(tmem_base_sm + 4);  // [kP1GatherWarps][128]
+  int32_t* tok_tab = reinterpret_cast<int32_t*>(tmem_base_sm + 4);  // [kGatherWarps][128] token of each row
 
   constexpr int kNumAcc = kFp8 ? 1 : 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -165,12 +183,14 @@ __global__ void __launch_bounds__(kP1Threads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1 + 32);  // TMA producer + the 32 lanes of one gather warp
+      // producer lane 0 (with the TMA byte count) + the cp.async completion
+      // arrivals of every gather lane
+      mbar_init(&full[s], 1 + 32 * kGatherWarps);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], kEpiWarps);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -192,15 +212,12 @@ __global__ void __launch_bounds__(kP1Threads, 1)
   const int esize = kFp8 ? 1 : 2;
 
   auto stage_ptr = [&](int s) { return smem + static_cast<size_t>(s) * p.stage_bytes; };
-  // stage layout: [A gate 16K][A up 16K][B bm*128][SFA gate 512][SFA up 512][SFB 512]
-  const int off_b = 2 * kTile * kRowBytes;
-  const int off_sf = off_b + p.bm * kRowBytes;
 
   if (warp == 0) {
-    // ------------------------------------------------ TMA producer
+    // ------------------------------------------------ TMA producer (weights)
     const uint64_t pol = policy_evict_first();
-    const uint32_t tx = 2 * kTile * kRowBytes + (kFp8 ? 2 * kSfTileBytes : 0);
-    const int MT1 = p.N / kTile, KT1 = p.K / 128;
+    const uint32_t tx = 2 * 128 * kRowBytes + (kFp8 ? 2 * kSfTileBytes : 0);
+    const int MT1 = p.N / 128, KT1 = p.K / 128;
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -208,22 +225,22 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       const int b = u / p.n_jt, j = u - (u / p.n_jt) * p.n_jt;
       const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
       if (bi.nend == 0) continue;
-      const int gate_row = bi.e * p.N + j * kTile;
-      const int up_row = bi.e * p.N + p.I + j * kTile;
+      const int gate_row = bi.e * p.N + j * kTI;
+      const int up_row = bi.e * p.N + p.I + j * kTI;
       for (int kc = 0; kc < n_kc; ++kc) {
         if (lane == 0) {
           ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
           if (ok) {
             uint8_t* st = stage_ptr(s);
             mbar_arrive_expect_tx(&full[s], tx);
-            tma_load_2d(st, &tm_w1, &full[s], kc * kKC, gate_row, pol);
-            tma_load_2d(st + kTile * kRowBytes, &tm_w1, &full[s], kc * kKC, up_row, pol);
+            tma_load_2d(st + kOffB, &tm_w1, &full[s], kc * kKC, gate_row, pol);
+            tma_load_2d(st + kOffB + 128 * kRowBytes, &tm_w1, &full[s], kc * kKC, up_row, pol);
             if (kFp8) {
               const uint8_t* sfg = p.w1_sf + ((static_cast<int64_t>(bi.e) * MT1 + j) * KT1 + kc) * kSfTileBytes;
               const uint8_t* sfu =
-                  p.w1_sf + ((static_cast<int64_t>(bi.e) * MT1 + p.I / kTile + j) * KT1 + kc) * kSfTileBytes;
-              bulk_load(st + off_sf, sfg, kSfTileBytes, &full[s]);
-              bulk_load(st + off_sf + kSfTileBytes, sfu, kSfTileBytes, &full[s]);
+                  p.w1_sf + ((static_cast<int64_t>(bi.e) * MT1 + p.I / 128 + j) * KT1 + kc) * kSfTileBytes;
+              bulk_load(st + kOffSf + kSfTileBytes, sfg, kSfTileBytes, &full[s]);
+              bulk_load(st + kOffSf + 2 * kSfTileBytes, sfu, kSfTileBytes, &full[s]);
             }
           }
         }
@@ -234,6 +251,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdesc = kFp8 ? 0u : idesc_bf16(kM, 256);
     int s = 0;
     uint32_t ph = 0;
     int acc_it = 0;
@@ -248,36 +266,33 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t d_gate = tbase + static_cast<uint32_t>(buf) * 256u;
-      const uint32_t d_up = d_gate + 128u;
+      const uint32_t d = tbase + static_cast<uint32_t>(buf) * 256u;
       for (int kc = 0; kc < n_kc; ++kc) {
         if (lane == 0) {
           ok = mbar_wait(&full[s], ph, abort_flag, p.status);
           if (ok) {
             tc_fence_after();
+            // the token rows (and scales) arrived through cp.async (generic
+            // proxy); the MMA and tcgen05.cp read them through the async proxy
+            fence_proxy_async_smem();
             uint8_t* st = stage_ptr(s);
-            const uint64_t ag = sdesc_sw128(smem_u32(st));
-            const uint64_t au = sdesc_sw128(smem_u32(st + kTile * kRowBytes));
-            const uint64_t bd = sdesc_sw128(smem_u32(st + off_b));
+            const uint64_t ad = sdesc_sw128(smem_u32(st));
+            const uint64_t bd = sdesc_sw128(smem_u32(st + kOffB));
             if (kFp8) {
-              tc_cp_32x128b_x4(tbase + kP1SfCol + 0, sdesc_sf(smem_u32(st + off_sf)));
-              tc_cp_32x128b_x4(tbase + kP1SfCol + 4, sdesc_sf(smem_u32(st + off_sf + kSfTileBytes)));
-              tc_cp_32x128b_x4(tbase + kP1SfCol + 8, sdesc_sf(smem_u32(st + off_sf + 2 * kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + kSfaCol, sdesc_sf(smem_u32(st + kOffSf)));
+              tc_cp_32x128b_x4(tbase + kSfbCol, sdesc_sf(smem_u32(st + kOffSf + kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + kSfbCol + 4, sdesc_sf(smem_u32(st + kOffSf + 2 * kSfTileBytes)));
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint32_t acc = (kc | kk) != 0;
               const uint64_t step = static_cast<uint64_t>(2 * kk);  // 32 bytes along K
               if (kFp8) {
-                const uint32_t id = idesc_mxf8(kTile, bi.n16, kk, kk);
                 const uint32_t sfid = static_cast<uint32_t>(kk) << 30;
-                const uint32_t sfb = (tbase + kP1SfCol + 8) | sfid;
-                mma_mxf8(d_gate, ag + step, bd + step, id, (tbase + kP1SfCol + 0) | sfid, sfb, acc);
-                mma_mxf8(d_up, au + step, bd + step, id, (tbase + kP1SfCol + 4) | sfid, sfb, acc);
+                mma_mxf8(d, ad + step, bd + step, idesc_mxf8(kM, 256, kk, kk), (tbase + kSfaCol) | sfid,
+                         (tbase + kSfbCol) | sfid, acc);
               } else {
-                const uint32_t id = idesc_bf16(kTile, bi.n16);
-                mma_f16(d_gate, ag + step, bd + step, id, acc);
-                mma_f16(d_up, au + step, bd + step, id, acc);
+                mma_f16(d, ad + step, bd + step, kIdesc, acc);
               }
             }
             tc_commit(&empty[s]);
@@ -290,14 +305,15 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       if (ok && lane == 0) tc_commit(&acc_full[buf]);
       ++acc_it;
     }
-  } else if (warp < 2 + kP1GatherWarps) {
+  } else if (warp < kP1FirstEpi) {
     // ------------------------------------------------ token gather
+    // Gather warp g copies the 16-row groups r0 = 16 (g + kGatherWarps i) of
+    // the block (and their token scales) for every stage, then lets the stage's
+    // mbarrier track the copies (cp.async.mbarrier.arrive) instead of
+    // waiting for them.  Rows past the block's last routed row are not
+    // loaded: the accumulator rows they produce are never read.
     const int g = warp - 2;
     int32_t* tok = tok_tab + g * 128;
-    // Gather warp g owns the stages s with s % kP1GatherWarps == g and fills
-    // every use of them in order, so its wait on empty[s] is never more than
-    // one phase behind the barrier (a parity wait cannot tell phase n from
-    // phase n + 2).
     const int KS = p.K / 32;
     int s = 0;
     uint32_t ph = 0;
@@ -306,53 +322,44 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       const int b = u / p.n_jt;
       const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
       if (bi.nend == 0) continue;
-      bool tok_ready = false;
+      __syncwarp();
+      for (int r = lane; r < bi.nend; r += 32)
+        tok[r] = row_valid(bi, r) ? __ldg(p.sorted_ids + static_cast<int64_t>(b) * p.bm + r) / p.top_k : -1;
+      __syncwarp();
       for (int kc = 0; kc < n_kc; ++kc) {
-        if (s % kP1GatherWarps == g) {
-          if (!tok_ready) {
-            __syncwarp();
-            for (int r = lane; r < bi.n16; r += 32) {
-              const int id = __ldg(p.sorted_ids + static_cast<int64_t>(b) * p.bm + r);
-              tok[r] = row_valid(bi, r) ? id / p.top_k : -1;
-            }
-            __syncwarp();
-            tok_ready = true;
+        if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        uint8_t* st = stage_ptr(s);
+        const uint32_t abase = smem_u32(st);
+        const uint32_t sfa = smem_u32(st + kOffSf);
+        for (int r0 = 16 * g; r0 < bi.nend; r0 += 16 * kGatherWarps) {
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {  // 16 rows x 8 chunks of 16 bytes
+            const int idx = 32 * it + lane;
+            const int r = r0 + (idx >> 3), q = idx & 7;
+            const int t = r < bi.nend ? tok[r] : -1;
+            if (t >= 0)
+              cp_async_16(abase + r * kRowBytes + ((q ^ (r & 7)) << 4),
+                          p.x + (static_cast<int64_t>(t) * p.K * esize + kc * kRowBytes + q * 16));
           }
-          if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) break;
-          uint8_t* st = stage_ptr(s);
-          const uint32_t bsm = smem_u32(st + off_b);
-          for (int idx = lane; idx < bi.n16 * 8; idx += 32) {
-            const int r = idx >> 3, q = idx & 7;
-            const uint32_t dst = bsm + r * kRowBytes + ((q ^ (r & 7)) << 4);
-            const int t = tok[r];
-            if (t >= 0) {
-              cp_async_16(dst, p.x + (static_cast<int64_t>(t) * p.K * esize + kc * kRowBytes + q * 16));
-            } else {
-              asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
-            }
+          if (kFp8 && lane < 16) {
+            const int r = r0 + lane;
+            const int t = r < bi.nend ? tok[r] : -1;
+            if (t >= 0) cp_async_4(sfa + (r & 31) * 16 + (r >> 5) * 4, p.x_sf + static_cast<int64_t>(t) * KS + 4 * kc);
           }
-          if (kFp8) {
-            uint8_t* sfb = st + off_sf + 2 * kSfTileBytes;
-            for (int r = lane; r < bi.n16; r += 32) {
-              const int t = tok[r];
-              uint32_t v = 0;
-              if (t >= 0) v = __ldg(reinterpret_cast<const uint32_t*>(p.x_sf + static_cast<int64_t>(t) * KS) + kc);
-              *reinterpret_cast<uint32_t*>(sfb + (r & 31) * 16 + (r >> 5) * 4) = v;
-            }
-          }
-          cp_async_commit();
-          cp_async_wait_all();
-          fence_proxy_async_smem();
-          mbar_arrive(&full[s]);
         }
+        cp_async_mbar_arrive(&full[s]);
         if (++s == S) { s = 0; ph ^= 1u; }
       }
     }
   } else {
-    // ------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quadrant of this warp
+    // ------------------------------------------------ epilogue (8 warps)
+    // Warp w reads TMEM lane quadrant w % 4 (rows 32q..32q+31, one per
+    // thread) and intermediate columns [64h, 64h + 64) of the unit's tile.
+    const int q = warp & 3;
+    const int h = (warp - kP1FirstEpi) >> 2;
+    const int r = 32 * q + lane;
     int acc_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -365,32 +372,54 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
+      const bool mine = row_valid(bi, r);
+      const int64_t row = static_cast<int64_t>(b) * p.bm + r;
       const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 256u;
-      const int icol = j * kTile + 32 * q + lane;
-      const int64_t row0 = static_cast<int64_t>(b) * p.bm;
-      for (int c0 = 0; c0 < bi.nend; c0 += 16) {
-        uint32_t gr[16], ur[16];
-        tmem_ld16(tacc + c0, gr);
-        tmem_ld16(tacc + 128 + c0, ur);
-        tmem_ld_wait();
+      if (32 * q < bi.nend) {  // warp-uniform: skip quadrants with no routed row
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          const int col0 = 64 * h + 32 * c;  // within the unit's 128-column tile
+          uint32_t gr[32], ur[32];
+          tmem_ld32(tacc + col0, gr);
+          tmem_ld32(tacc + 128 + col0, ur);
+          tmem_ld_wait();
+          float a[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = c0 + i;
-          const float a = silu_f32(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
+          for (int i = 0; i < 32; ++i) a[i] = silu_f32(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
+          const int icol = j * kTI + col0;
           if (kFp8) {
-            const uint32_t amax_bits = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(a)));
-            int sc = static_cast<int>((amax_bits >> 23) & 0xFFu) - 127 - 8;
+            float amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(a[i]));
+            int sc = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127 - 8;
             sc = sc < -127 ? -127 : (sc > 127 ? 127 : sc);
             const float inv = __uint_as_float(static_cast<uint32_t>(127 - sc) << 23);
-            if (row_valid(bi, c)) {
-              p.act[(row0 + c) * p.I + icol] = static_cast<uint8_t>(cvt_e4m3x2(a * inv, 0.0f) & 0xFFu);
-              if (lane == 0)
-                p.act_sf[(static_cast<int64_t>(b) * p.n_jt + j) * kSfTileBytes + (c & 31) * 16 + (c >> 5) * 4 + q] =
-                    static_cast<uint8_t>(sc + 127);
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              w[i] = static_cast<uint32_t>(cvt_e4m3x2(a[4 * i] * inv, a[4 * i + 1] * inv)) |
+                     (static_cast<uint32_t>(cvt_e4m3x2(a[4 * i + 2] * inv, a[4 * i + 3] * inv)) << 16);
+            if (mine) {
+              uint4* dst = reinterpret_cast<uint4*>(p.act + row * p.I + icol);
+              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+              p.act_sf[(static_cast<int64_t>(b) * p.n_jt + j) * kSfTileBytes + (r & 31) * 16 + (r >> 5) * 4 +
+                       (col0 >> 5)] = static_cast<uint8_t>(sc + 127);
             }
-          } else {
-            if (row_valid(bi, c) && icol < p.I)
-              reinterpret_cast<__nv_bfloat16*>(p.act)[(row0 + c) * p.I + icol] = __float2bfloat16_rn(a);
+          } else if (mine && icol < p.I) {
+            __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.act) + row * p.I + icol;
+            if (icol + 32 <= p.I) {
+              uint32_t w[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(a[2 * i], a[2 * i + 1]);
+              uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (icol + i < p.I) dst[i] = __float2bfloat16_rn(a[i]);
+            }
           }
         }
       }
@@ -428,7 +457,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
   uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sm + 1);
 
-  constexpr int kNumAcc = 2;
+  constexpr int kNumAcc = kFp8 ? 1 : 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -437,7 +466,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 4);
+      mbar_init(&acc_empty[a], kEpiWarps);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -457,15 +486,12 @@ __global__ void __launch_bounds__(kP2Threads, 1)
   const int n_units = n_blocks * p.n_ht;
   constexpr int kKC = kFp8 ? 128 : 64;
   auto stage_ptr = [&](int s) { return smem + static_cast<size_t>(s) * p.stage_bytes; };
-  // stage layout: [A (w2 rows) 16K][B (intermediate rows) bm*128][SFA 512][SFB 512]
-  const int off_b = kTile * kRowBytes;
-  const int off_sf = off_b + p.bm * kRowBytes;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_a = policy_evict_last();
-    const int MT2 = p.K / kTile, KT2 = p.I / 128;
+    const int MT2 = p.K / 128, KT2 = p.I / 128;
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -473,22 +499,26 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       const int b = u / p.n_ht, ht = u - (u / p.n_ht) * p.n_ht;
       const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
       if (bi.nend == 0) continue;
-      const int w2_row = bi.e * p.K + ht * kTile;
-      const uint32_t tx = kTile * kRowBytes + bi.n16 * kRowBytes + (kFp8 ? 2 * kSfTileBytes : 0);
+      const int nb = min(2, (p.K - ht * kTH) / 128);  // 128-row halves of this feature tile
+      const int w2_row = bi.e * p.K + ht * kTH;
+      const uint32_t tx = nb * 128 * kRowBytes + bi.n16 * kRowBytes + (kFp8 ? (1 + nb) * kSfTileBytes : 0);
       for (int kc = 0; kc < p.n_kc; ++kc) {
         if (lane == 0) {
           ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
           if (ok) {
             uint8_t* st = stage_ptr(s);
             mbar_arrive_expect_tx(&full[s], tx);
-            tma_load_2d(st, &tm_w2, &full[s], kc * kKC, w2_row, pol_w);
             for (int i = 0; i < bi.n16 / 16; ++i)
-              tma_load_2d(st + off_b + i * 16 * kRowBytes, &tm_act, &full[s], kc * kKC, b * p.bm + 16 * i, pol_a);
+              tma_load_2d(st + i * 16 * kRowBytes, &tm_act, &full[s], kc * kKC, b * p.bm + 16 * i, pol_a);
+            for (int i = 0; i < nb; ++i)
+              tma_load_2d(st + kOffB + i * 128 * kRowBytes, &tm_w2, &full[s], kc * kKC, w2_row + 128 * i, pol_w);
             if (kFp8) {
-              const uint8_t* sfa = p.w2_sf + ((static_cast<int64_t>(bi.e) * MT2 + ht) * KT2 + kc) * kSfTileBytes;
-              const uint8_t* sfb = p.act_sf + (static_cast<int64_t>(b) * KT2 + kc) * kSfTileBytes;
-              bulk_load(st + off_sf, sfa, kSfTileBytes, &full[s]);
-              bulk_load(st + off_sf + kSfTileBytes, sfb, kSfTileBytes, &full[s]);
+              bulk_load(st + kOffSf, p.act_sf + (static_cast<int64_t>(b) * KT2 + kc) * kSfTileBytes, kSfTileBytes,
+                        &full[s]);
+              for (int i = 0; i < nb; ++i)
+                bulk_load(st + kOffSf + (1 + i) * kSfTileBytes,
+                          p.w2_sf + ((static_cast<int64_t>(bi.e) * MT2 + 2 * ht + i) * KT2 + kc) * kSfTileBytes,
+                          kSfTileBytes, &full[s]);
             }
           }
         }
@@ -504,16 +534,17 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     int acc_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int b = u / p.n_ht;
+      const int b = u / p.n_ht, ht = u - (u / p.n_ht) * p.n_ht;
       const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
       if (bi.nend == 0) continue;
+      const int nn = min(kTH, p.K - ht * kTH);
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
       if (lane == 0) ok = mbar_wait(&acc_empty[buf], acc_ph ^ 1u, abort_flag, p.status);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t d = tbase + static_cast<uint32_t>(buf) * 128u;
+      const uint32_t d = tbase + static_cast<uint32_t>(buf) * 256u;
       for (int kc = 0; kc < p.n_kc; ++kc) {
         if (lane == 0) {
           ok = mbar_wait(&full[s], ph, abort_flag, p.status);
@@ -521,10 +552,11 @@ __global__ void __launch_bounds__(kP2Threads, 1)
             tc_fence_after();
             uint8_t* st = stage_ptr(s);
             const uint64_t ad = sdesc_sw128(smem_u32(st));
-            const uint64_t bd = sdesc_sw128(smem_u32(st + off_b));
+            const uint64_t bd = sdesc_sw128(smem_u32(st + kOffB));
             if (kFp8) {
-              tc_cp_32x128b_x4(tbase + kP2SfCol + 0, sdesc_sf(smem_u32(st + off_sf)));
-              tc_cp_32x128b_x4(tbase + kP2SfCol + 4, sdesc_sf(smem_u32(st + off_sf + kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + kSfaCol, sdesc_sf(smem_u32(st + kOffSf)));
+              tc_cp_32x128b_x4(tbase + kSfbCol, sdesc_sf(smem_u32(st + kOffSf + kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + kSfbCol + 4, sdesc_sf(smem_u32(st + kOffSf + 2 * kSfTileBytes)));
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -532,10 +564,10 @@ __global__ void __launch_bounds__(kP2Threads, 1)
               const uint64_t step = static_cast<uint64_t>(2 * kk);
               if (kFp8) {
                 const uint32_t sfid = static_cast<uint32_t>(kk) << 30;
-                mma_mxf8(d, ad + step, bd + step, idesc_mxf8(kTile, bi.n16, kk, kk), (tbase + kP2SfCol) | sfid,
-                         (tbase + kP2SfCol + 4) | sfid, acc);
+                mma_mxf8(d, ad + step, bd + step, idesc_mxf8(kM, nn, kk, kk), (tbase + kSfaCol) | sfid,
+                         (tbase + kSfbCol) | sfid, acc);
               } else {
-                mma_f16(d, ad + step, bd + step, idesc_bf16(kTile, bi.n16), acc);
+                mma_f16(d, ad + step, bd + step, idesc_bf16(kM, nn), acc);
               }
             }
             tc_commit(&empty[s]);
@@ -549,37 +581,52 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       ++acc_it;
     }
   } else {
-    // ------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------ epilogue (8 warps)
+    // Warp w reads TMEM lane quadrant w % 4 (rows 32q..32q+31, one per
+    // thread) and half h of the unit's output features.
     const int q = warp & 3;
+    const int h = (warp - kP2FirstEpi) >> 2;
+    const int r = 32 * q + lane;
     int acc_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
       const int b = u / p.n_ht, ht = u - (u / p.n_ht) * p.n_ht;
       const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
       if (bi.nend == 0) continue;
+      const int nn = min(kTH, p.K - ht * kTH);
+      const int64_t row0 = static_cast<int64_t>(b) * p.bm;
+      // the route and its weight, fetched while the MMAs run
+      const bool mine = row_valid(bi, r);
+      int route = 0;
+      float wgt = 0.f;
+      if (mine) {
+        route = __ldg(p.sorted_ids + row0 + r);
+        wgt = __ldg(p.topk_w + route);
+      }
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
       ok = mbar_wait(&acc_full[buf], acc_ph, abort_flag, p.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 128u;
-      const int hcol = ht * kTile + 32 * q + lane;
-      const int64_t row0 = static_cast<int64_t>(b) * p.bm;
-      for (int c0 = 0; c0 < bi.nend; c0 += 16) {
-        uint32_t yr[16];
-        tmem_ld16(tacc + c0, yr);
-        tmem_ld_wait();
+      const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 256u;
+      if (32 * q < bi.nend) {
+        const int half = nn / 2;
+        float* dst = p.yw + static_cast<int64_t>(route) * p.K + ht * kTH + h * half;
+#pragma unroll 1
+        for (int c = 0; c < half; c += 32) {
+          uint32_t yr[32];
+          tmem_ld32(tacc + h * half + c, yr);
+          tmem_ld_wait();
+          if (mine) {
+            float4* d4 = reinterpret_cast<float4*>(dst + c);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = c0 + i;
-          if (row_valid(bi, c)) {
-            const int route = __ldg(p.sorted_ids + row0 + c);
-            const float w = __ldg(p.topk_w + route);
-            p.yw[static_cast<int64_t>(route) * p.K + hcol] = w * __uint_as_float(yr[i]);
-            if (ht == 0 && q == 0 && lane == 0) p.flags[route] = 1;
+            for (int i = 0; i < 8; ++i)
+              d4[i] = make_float4(wgt * __uint_as_float(yr[4 * i]), wgt * __uint_as_float(yr[4 * i + 1]),
+                                  wgt * __uint_as_float(yr[4 * i + 2]), wgt * __uint_as_float(yr[4 * i + 3]));
           }
         }
+        if (mine && ht == 0 && h == 0) p.flags[route] = 1;
       }
       tc_fence_before();
       __syncwarp();
@@ -723,13 +770,10 @@ struct FusedArgs {
   cudaStream_t stream;
 };
 
-static int p1_stage_bytes(bool fp8, int bm) {
-  return static_cast<int>(round_up(2 * kTile * kRowBytes + bm * kRowBytes + (fp8 ? 3 * kSfTileBytes : 0), 1024));
+static int stage_bytes(bool fp8) {
+  return static_cast<int>(round_up(kOffSf + (fp8 ? 3 * kSfTileBytes : 0), 1024));
 }
-static int p2_stage_bytes(bool fp8, int bm) {
-  return static_cast<int>(round_up(kTile * kRowBytes + bm * kRowBytes + (fp8 ? 2 * kSfTileBytes : 0), 1024));
-}
-constexpr int kP1Ctrl = 64 * 16 + 16 + kP1GatherWarps * 128 * 4;  // barriers, tmem base, flags, token tables
+constexpr int kP1Ctrl = 64 * 16 + 16 + kGatherWarps * 128 * 4;  // barriers, tmem base, flags, token tables
 constexpr int kP2Ctrl = 64 * 16 + 16;
 
 static int pick_stages(int stage_bytes, int ctrl, int requested, int max_stages) {
@@ -785,8 +829,8 @@ static int run_fused(const FusedArgs& a) {
 
   CUtensorMap tm_w1, tm_w2, tm_act;
   int rc;
-  if ((rc = make_tmap(&tm_w1, a.w1, a.fp8, static_cast<int64_t>(a.E) * a.N, a.K, kTile)) != MOE_OK) return rc;
-  if ((rc = make_tmap(&tm_w2, a.w2, a.fp8, static_cast<int64_t>(a.E) * a.K, I, kTile)) != MOE_OK) return rc;
+  if ((rc = make_tmap(&tm_w1, a.w1, a.fp8, static_cast<int64_t>(a.E) * a.N, a.K, 128)) != MOE_OK) return rc;
+  if ((rc = make_tmap(&tm_w2, a.w2, a.fp8, static_cast<int64_t>(a.E) * a.K, I, 128)) != MOE_OK) return rc;
   if ((rc = make_tmap(&tm_act, ws + L.act, a.fp8, L.cap_rows, I, 16)) != MOE_OK) return rc;
 
   const int nsm = sm_count();
@@ -811,8 +855,8 @@ static int run_fused(const FusedArgs& a) {
   p1.K = a.K; p1.N = a.N; p1.I = I; p1.E = a.E; p1.top_k = a.top_k; p1.bm = a.bm;
   p1.R = a.T * a.top_k;
   p1.max_blocks = max_blocks;
-  p1.n_jt = (I + kTile - 1) / kTile;
-  p1.stage_bytes = p1_stage_bytes(a.fp8, a.bm);
+  p1.n_jt = (I + kTI - 1) / kTI;
+  p1.stage_bytes = stage_bytes(a.fp8);
   p1.stages = pick_stages(p1.stage_bytes, kP1Ctrl, req_stages, 8);
 
   P2Params p2{};
@@ -827,9 +871,9 @@ static int run_fused(const FusedArgs& a) {
   p2.status = p1.status;
   p2.K = a.K; p2.I = I; p2.E = a.E; p2.top_k = a.top_k; p2.bm = a.bm; p2.R = p1.R;
   p2.max_blocks = max_blocks;
-  p2.n_ht = a.K / kTile;
+  p2.n_ht = (a.K + kTH - 1) / kTH;
   p2.n_kc = a.fp8 ? I / 128 : (I + 63) / 64;
-  p2.stage_bytes = p2_stage_bytes(a.fp8, a.bm);
+  p2.stage_bytes = stage_bytes(a.fp8);
   p2.stages = pick_stages(p2.stage_bytes, kP2Ctrl, req_stages, 8);
   if (p1.stages < 2 || p2.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "%s: shared memory too small", nm);
 
