@@ -20,10 +20,10 @@
 //            codes all stay in its registers, and the intermediate row segment
 //            is written with 16-byte stores into an L2-resident workspace.
 //            Warp roles: 0 TMA producer (weight tiles, weight scale tiles),
-//            1 MMA issuer, 2-3 token gather (cp.async of the routed rows and,
+//            1 MMA issuer, 2-5 token gather (cp.async of the routed rows and,
 //            on mxfp8, their scales; completion is tracked by the stage's
 //            mbarrier, so the gather warps never wait on their own copies),
-//            4-11 epilogue (two warps per TMEM lane quadrant, one per column
+//            6-13 epilogue (two warps per TMEM lane quadrant, one per column
 //            half).
 //   phase 2  persistent kernel, unit = (block b, 256 output features).  A =
 //            the block's intermediate rows (TMA), B = 256 rows of w2[e] (TMA),
@@ -56,9 +56,10 @@ constexpr uint32_t kSfaCol = 256;   // 4 columns: 128 rows of A
 constexpr uint32_t kSfbCol = 260;   // 8 columns: 256 rows of B
 
 constexpr int kEpiWarps = 8;
-constexpr int kGatherWarps = 2;
+constexpr int kGatherWarps = 4;
+constexpr int kGatherSlots = 128 * 8 / (32 * kGatherWarps);  // 16-byte row chunks per gather lane and stage
 constexpr int kP1FirstEpi = 2 + kGatherWarps;
-constexpr int kP1Threads = 32 * (kP1FirstEpi + kEpiWarps);  // 12 warps
+constexpr int kP1Threads = 32 * (kP1FirstEpi + kEpiWarps);  // 14 warps
 constexpr int kP2FirstEpi = 2;
 constexpr int kP2Threads = 32 * (kP2FirstEpi + kEpiWarps);  // 10 warps
 
@@ -173,7 +174,6 @@ __global__ void __launch_bounds__(kP1Threads, 1)
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_base_sm = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sm + 1);
-  int32_t* tok_tab = reinterpret_cast<int32_t*>(tmem_base_sm + 4);  // [kGatherWarps][128] token of each row
 
   constexpr int kNumAcc = kFp8 ? 1 : 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -307,14 +307,18 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     }
   } else if (warp < kP1FirstEpi) {
     // ------------------------------------------------ token gather
-    // Gather warp g copies the 16-row groups r0 = 16 (g + kGatherWarps i) of
-    // the block (and their token scales) for every stage, then lets the stage's
-    // mbarrier track the copies (cp.async.mbarrier.arrive) instead of
-    // waiting for them.  Rows past the block's last routed row are not
-    // loaded: the accumulator rows they produce are never read.
+    // The 128 rows x 8 chunks of 16 bytes of a stage's A tile are dealt out
+    // once per unit: lane l of gather warp g owns chunk q = l % 8 of rows
+    // 4 g + 16 i + l / 8 (i < kGatherSlots), and on mxfp8 the 4-byte token
+    // scale of row 32 g + l.  Source addresses are computed once per unit,
+    // so a stage costs each lane a handful of independent cp.async; the
+    // stage's mbarrier tracks their completion (cp.async.mbarrier.arrive),
+    // so the gather warps never wait on their own copies.  Rows past the
+    // block's last routed row are not loaded: the accumulator rows they
+    // produce are never read.
     const int g = warp - 2;
-    int32_t* tok = tok_tab + g * 128;
     const int KS = p.K / 32;
+    const int q = lane & 7;
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
@@ -322,33 +326,37 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       const int b = u / p.n_jt;
       const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
       if (bi.nend == 0) continue;
-      __syncwarp();
-      for (int r = lane; r < bi.nend; r += 32)
-        tok[r] = row_valid(bi, r) ? __ldg(p.sorted_ids + static_cast<int64_t>(b) * p.bm + r) / p.top_k : -1;
-      __syncwarp();
+      const int64_t row0 = static_cast<int64_t>(b) * p.bm;
+      const uint8_t* src[kGatherSlots];
+      uint32_t dst[kGatherSlots];
+      uint32_t live = 0;
+#pragma unroll
+      for (int i = 0; i < kGatherSlots; ++i) {
+        const int r = 4 * g + 16 * i + (lane >> 3);
+        dst[i] = static_cast<uint32_t>(r * kRowBytes + ((q ^ (r & 7)) << 4));
+        src[i] = p.x;
+        if (r < bi.nend && row_valid(bi, r)) {
+          const int t = __ldg(p.sorted_ids + row0 + r) / p.top_k;
+          src[i] = p.x + static_cast<int64_t>(t) * p.K * esize + q * 16;
+          live |= 1u << i;
+        }
+      }
+      const uint8_t* sf_src = nullptr;
+      const uint32_t sf_dst = static_cast<uint32_t>((lane & 31) * 16 + g * 4);  // row r = 32 g + lane
+      if (kFp8) {
+        const int r = 32 * g + lane;
+        if (r < bi.nend && row_valid(bi, r))
+          sf_src = p.x_sf + static_cast<int64_t>(__ldg(p.sorted_ids + row0 + r) / p.top_k) * KS;
+      }
       for (int kc = 0; kc < n_kc; ++kc) {
         if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
-        uint8_t* st = stage_ptr(s);
-        const uint32_t abase = smem_u32(st);
-        const uint32_t sfa = smem_u32(st + kOffSf);
-        for (int r0 = 16 * g; r0 < bi.nend; r0 += 16 * kGatherWarps) {
+        const uint32_t abase = smem_u32(stage_ptr(s));
 #pragma unroll
-          for (int it = 0; it < 4; ++it) {  // 16 rows x 8 chunks of 16 bytes
-            const int idx = 32 * it + lane;
-            const int r = r0 + (idx >> 3), q = idx & 7;
-            const int t = r < bi.nend ? tok[r] : -1;
-            if (t >= 0)
-              cp_async_16(abase + r * kRowBytes + ((q ^ (r & 7)) << 4),
-                          p.x + (static_cast<int64_t>(t) * p.K * esize + kc * kRowBytes + q * 16));
-          }
-          if (kFp8 && lane < 16) {
-            const int r = r0 + lane;
-            const int t = r < bi.nend ? tok[r] : -1;
-            if (t >= 0) cp_async_4(sfa + (r & 31) * 16 + (r >> 5) * 4, p.x_sf + static_cast<int64_t>(t) * KS + 4 * kc);
-          }
-        }
+        for (int i = 0; i < kGatherSlots; ++i)
+          if (live & (1u << i)) cp_async_16(abase + dst[i], src[i] + kc * kRowBytes);
+        if (kFp8 && sf_src) cp_async_4(abase + kOffSf + sf_dst, sf_src + 4 * kc);
         cp_async_mbar_arrive(&full[s]);
         if (++s == S) { s = 0; ph ^= 1u; }
       }
@@ -773,7 +781,7 @@ struct FusedArgs {
 static int stage_bytes(bool fp8) {
   return static_cast<int>(round_up(kOffSf + (fp8 ? 3 * kSfTileBytes : 0), 1024));
 }
-constexpr int kP1Ctrl = 64 * 16 + 16 + kGatherWarps * 128 * 4;  // barriers, tmem base, flags, token tables
+constexpr int kP1Ctrl = 64 * 16 + 16;  // barriers, tmem base, abort flag
 constexpr int kP2Ctrl = 64 * 16 + 16;
 
 static int pick_stages(int stage_bytes, int ctrl, int requested, int max_stages) {
