@@ -63,6 +63,12 @@ constexpr int kP1Threads = 32 * (kP1FirstEpi + kEpiWarps);  // 14 warps
 constexpr int kP2FirstEpi = 2;
 constexpr int kP2Threads = 32 * (kP2FirstEpi + kEpiWarps);  // 10 warps
 
+// Control area after the stages: mbarriers, TMEM base, abort flag; in
+// phase 2 followed by each epilogue warp's 32 x 16 fp32 store staging.
+constexpr int kP2Ctrl = 64 * 16 + 16;
+constexpr int kStageFloatsPerWarp = 32 * 16;
+constexpr int kP2Staging = kEpiWarps * kStageFloatsPerWarp * 4;
+
 // Stage layout (both phases): [A 128 rows x 128 B][B 256 rows x 128 B][SFA 512][SFB 2 x 512]
 constexpr int kOffB = kM * kRowBytes;
 constexpr int kOffSf = kOffB + 2 * 128 * kRowBytes;
@@ -595,6 +601,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     const int q = warp & 3;
     const int h = (warp - kP2FirstEpi) >> 2;
     const int r = 32 * q + lane;
+    float4* stg4 = reinterpret_cast<float4*>(ctrl + kP2Ctrl) + (warp - kP2FirstEpi) * (kStageFloatsPerWarp / 4);
     int acc_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -619,19 +626,38 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       tc_fence_after();
       const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 256u;
       if (32 * q < bi.nend) {
+        // Thread = row.  Each 16-column slice of the warp's 32 rows goes
+        // through shared memory so that the stores leave as 64 contiguous
+        // bytes per row (8 rows per instruction) instead of 16 bytes to 32
+        // different rows.  float4 slot i of row l sits at i ^ (l & 3).
         const int half = nn / 2;
-        float* dst = p.yw + static_cast<int64_t>(route) * p.K + ht * kTH + h * half;
+        const int64_t col_base = static_cast<int64_t>(ht) * kTH + h * half;
 #pragma unroll 1
         for (int c = 0; c < half; c += 32) {
           uint32_t yr[32];
           tmem_ld32(tacc + h * half + c, yr);
           tmem_ld_wait();
-          if (mine) {
-            float4* d4 = reinterpret_cast<float4*>(dst + c);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              d4[i] = make_float4(wgt * __uint_as_float(yr[4 * i]), wgt * __uint_as_float(yr[4 * i + 1]),
-                                  wgt * __uint_as_float(yr[4 * i + 2]), wgt * __uint_as_float(yr[4 * i + 3]));
+          for (int hh = 0; hh < 2; ++hh) {
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int k = 16 * hh + 4 * i;
+              stg4[lane * 4 + (i ^ (lane & 3))] =
+                  make_float4(wgt * __uint_as_float(yr[k]), wgt * __uint_as_float(yr[k + 1]),
+                              wgt * __uint_as_float(yr[k + 2]), wgt * __uint_as_float(yr[k + 3]));
+            }
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int rl = 8 * it + (lane >> 2), cq = lane & 3;
+              const float4 v = stg4[rl * 4 + (cq ^ (rl & 3))];
+              const int route_l = __shfl_sync(0xffffffffu, route, rl);
+              const int mine_l = __shfl_sync(0xffffffffu, static_cast<int>(mine), rl);
+              if (mine_l)
+                *reinterpret_cast<float4*>(p.yw + static_cast<int64_t>(route_l) * p.K + col_base + c + 16 * hh +
+                                           4 * cq) = v;
+            }
           }
         }
         if (mine && ht == 0 && h == 0) p.flags[route] = 1;
@@ -782,7 +808,6 @@ static int stage_bytes(bool fp8) {
   return static_cast<int>(round_up(kOffSf + (fp8 ? 3 * kSfTileBytes : 0), 1024));
 }
 constexpr int kP1Ctrl = 64 * 16 + 16;  // barriers, tmem base, abort flag
-constexpr int kP2Ctrl = 64 * 16 + 16;
 
 static int pick_stages(int stage_bytes, int ctrl, int requested, int max_stages) {
   int s = (kSmemLimit - 1024 - ctrl) / stage_bytes;
@@ -882,7 +907,7 @@ static int run_fused(const FusedArgs& a) {
   p2.n_ht = (a.K + kTH - 1) / kTH;
   p2.n_kc = a.fp8 ? I / 128 : (I + 63) / 64;
   p2.stage_bytes = stage_bytes(a.fp8);
-  p2.stages = pick_stages(p2.stage_bytes, kP2Ctrl, req_stages, 8);
+  p2.stages = pick_stages(p2.stage_bytes, kP2Ctrl + kP2Staging, req_stages, 8);
   if (p1.stages < 2 || p2.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "%s: shared memory too small", nm);
 
   const int64_t units1 = static_cast<int64_t>(max_blocks) * p1.n_jt;
@@ -893,7 +918,7 @@ static int run_fused(const FusedArgs& a) {
   // Each CTA allocates all 512 TMEM columns: request more than half of the
   // shared memory so that two CTAs never share an SM.
   const int smem1 = std::max(1024 + p1.stages * p1.stage_bytes + kP1Ctrl, kSmemLimit / 2 + 1024);
-  const int smem2 = std::max(1024 + p2.stages * p2.stage_bytes + kP2Ctrl, kSmemLimit / 2 + 1024);
+  const int smem2 = std::max(1024 + p2.stages * p2.stage_bytes + kP2Ctrl + kP2Staging, kSmemLimit / 2 + 1024);
 
   void* const* ev = a.tune ? a.tune->phase_events : nullptr;
   auto mark = [&](int i) -> int {
