@@ -182,6 +182,39 @@ MOE_API int fused_moe_mxfp8(const uint8_t* x_e4m3, const uint8_t* x_scales, cons
                     int block_m, int64_t capacity, void* workspace, int64_t workspace_bytes,
                     const moe_tuning* tune, moe_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * fused_moe_bf16_noalloc -- the pages have no counterpart to this call; it
+ * is a convenience of this library.  It computes exactly what
+ * fused_moe_bf16 computes, for callers that cannot allocate device memory
+ * for the workspace: a plain C host program that links only this library
+ * and has no device allocator of its own, or an application whose memory
+ * pool owns all device memory and forbids further cudaMalloc calls.
+ *
+ * The workspace is a file-scope device array of MOE_NOALLOC_SCRATCH_BYTES
+ * inside the library; every GPU that loads the library holds it until the
+ * process exits.  Problems whose moe_workspace_bytes(MOE_DTYPE_BF16, ...)
+ * exceeds that size are rejected with MOE_ERR_WORKSPACE before anything is
+ * launched (small batches fit; e.g. T=64, K=N=1024, E=8, top_k=2 needs
+ * about 1.2 MB, while E=256 experts with N=4096 need far more and must use
+ * fused_moe_bf16).  The call allocates nothing.
+ *
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture begins.
+ *   - All calls share the one array, which keeps the last call's contents;
+ *     nothing in it has to start at zero.  Calls whose kernels overlap on
+ *     the GPU (different streams, or different host threads) race on it and
+ *     must be serialised by the caller.
+ *   Arguments, constraints and errors otherwise as fused_moe_bf16.
+ * ---------------------------------------------------------------------- */
+#define MOE_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+MOE_API int64_t fused_moe_bf16_noalloc_max_workspace(void);
+MOE_API int fused_moe_bf16_noalloc(const void* x, const void* w1, const void* w2,
+                                   const int32_t* sorted_token_ids, const int32_t* expert_ids,
+                                   const int32_t* num_tokens_post_padded, const float* topk_weights,
+                                   void* out, int T, int K, int N, int E, int top_k, int block_m,
+                                   int64_t capacity, const moe_tuning* tune, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,7 +28,8 @@ from . import _build
 __all__ = [
     "MoeError", "load", "moe_align", "moe_align_capacity", "fused_moe_bf16", "fused_moe_mxfp8",
     "pack_scales_blocked", "pack_scales_blocked_bytes", "moe_workspace_bytes", "moe_device_status",
-    "Tuning", "DTYPE_BF16", "DTYPE_MXFP8", "LIB_PATH",
+    "Tuning", "DTYPE_BF16", "DTYPE_MXFP8", "LIB_PATH", "fused_moe_bf16_noalloc",
+    "fused_moe_bf16_noalloc_max_workspace",
 ]
 
 DTYPE_BF16 = 0
@@ -82,6 +83,8 @@ _SIGS = {
     "fused_moe_bf16": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _I64, _P, _P], _I),
     "fused_moe_mxfp8": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _I64,
                          _P, _P], _I),
+    "fused_moe_bf16_noalloc_max_workspace": ([], _I64),
+    "fused_moe_bf16_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _P], _I),
 }
 
 
@@ -255,6 +258,35 @@ def fused_moe_mxfp8(x, x_scales, w1, w1_scales_blocked, w2, w2_scales_blocked, s
         _ptr(x), _ptr(x_scales), _ptr(w1), _ptr(w1_scales_blocked), _ptr(w2), _ptr(w2_scales_blocked),
         _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(topk_weights), _ptr(out),
         T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws), ws.numel(),
+        None if tune is None else ctypes.byref(tune), _stream(stream)))
+    return out
+
+
+def fused_moe_bf16_noalloc_max_workspace() -> int:
+    """Size of the library-owned workspace used by fused_moe_bf16_noalloc."""
+    return int(load().fused_moe_bf16_noalloc_max_workspace())
+
+
+def fused_moe_bf16_noalloc(x, w1, w2, sorted_token_ids, expert_ids, num_tokens_post_padded, topk_weights, out,
+                           block_m: int, tune: Tuning | None = None, stream=None):
+    """fused_moe_bf16 without a caller workspace: uses the library's fixed-size
+    device scratch, so nothing is allocated.  For callers that cannot allocate
+    device memory; problems needing more than
+    fused_moe_bf16_noalloc_max_workspace() bytes are rejected."""
+    import torch
+
+    for t, n in ((x, "x"), (w1, "w1"), (w2, "w2"), (out, "out")):
+        _need(t, n, (torch.bfloat16,))
+    _need(topk_weights, "topk_weights", (torch.float32,))
+    for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
+                 (num_tokens_post_padded, "num_tokens_post_padded")):
+        _need(t, n, (torch.int32,))
+    T, K = x.shape
+    E, N, _ = w1.shape
+    top_k = topk_weights.shape[1]
+    _check(load().fused_moe_bf16_noalloc(
+        _ptr(x), _ptr(w1), _ptr(w2), _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded),
+        _ptr(topk_weights), _ptr(out), T, K, N, E, top_k, block_m, sorted_token_ids.numel(),
         None if tune is None else ctypes.byref(tune), _stream(stream)))
     return out
 

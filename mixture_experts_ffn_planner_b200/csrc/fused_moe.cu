@@ -1014,3 +1014,60 @@ extern "C" int fused_moe_mxfp8(const uint8_t* x_e4m3, const uint8_t* x_scales, c
   a.stream = reinterpret_cast<cudaStream_t>(stream);
   return run_fused(a);
 }
+
+// ========================================================================
+// fused_moe_bf16_noalloc: the bf16 forward with a library-owned workspace
+// ========================================================================
+namespace moe {
+
+// Some callers cannot allocate device memory for the workspace: a plain C
+// host program that links only this library and has no allocator of its
+// own, or an application whose memory pool owns every byte of the device
+// and forbids extra cudaMalloc calls.  For them the workspace lives in this
+// file-scope array, which every device that loads the library keeps for the
+// life of the process.
+constexpr int64_t kNoAllocScratchBytes = int64_t(MOE_NOALLOC_SCRATCH_BYTES);
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch, looked up once per device (host code
+// cannot use the array's name as a device pointer).
+static int noalloc_scratch(void** out) {
+  static void* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("fused_moe_bf16_noalloc: cudaGetDevice");
+  if (dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "fused_moe_bf16_noalloc: device index %d too large", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (err != cudaSuccess) return cuda_fail("fused_moe_bf16_noalloc: cudaGetSymbolAddress", err);
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" int64_t fused_moe_bf16_noalloc_max_workspace(void) { return moe::kNoAllocScratchBytes; }
+
+extern "C" int fused_moe_bf16_noalloc(const void* x, const void* w1, const void* w2,
+                                      const int32_t* sorted_token_ids, const int32_t* expert_ids,
+                                      const int32_t* num_tokens_post_padded, const float* topk_weights, void* out,
+                                      int T, int K, int N, int E, int top_k, int block_m, int64_t capacity,
+                                      const moe_tuning* tune, moe_stream_t stream) {
+  const int64_t need = moe_workspace_bytes(MOE_DTYPE_BF16, T, K, N, E, top_k, block_m);
+  if (need < 0)
+    return moe::fail(MOE_ERR_INVALID_ARG, "fused_moe_bf16_noalloc: invalid sizes");
+  if (need > moe::kNoAllocScratchBytes)
+    return moe::fail(MOE_ERR_WORKSPACE,
+                     "fused_moe_bf16_noalloc: this problem needs %lld bytes of workspace, more than the %lld-byte "
+                     "built-in scratch; use fused_moe_bf16 with a caller-allocated workspace",
+                     (long long)need, (long long)moe::kNoAllocScratchBytes);
+  void* ws = nullptr;
+  const int rc = moe::noalloc_scratch(&ws);
+  if (rc != MOE_OK) return rc;
+  return fused_moe_bf16(x, w1, w2, sorted_token_ids, expert_ids, num_tokens_post_padded, topk_weights, out, T, K, N,
+                        E, top_k, block_m, capacity, ws, moe::kNoAllocScratchBytes, tune, stream);
+}
