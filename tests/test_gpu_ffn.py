@@ -130,7 +130,8 @@ def test_c1_full():
     """bf16, T=64, K=1024, N=1024, E=8, top-2, block_m=64: whole oracle."""
     sh = W.shape("C1", 64)
     inp = W.inputs(sh)
-    check(sh, gpu_forward(sh, inp), oracle_forward(sh, inp), "C1")
+    rel, cos = check(sh, gpu_forward(sh, inp), oracle_forward(sh, inp), "C1")
+    print(f"PARITY C1 T=64 tokens=64 max|diff|/rms={rel:.3e} cos={cos:.7f}")
 
 
 @pytest.mark.parametrize("T", [1, 8, 64, 512, 8192])
@@ -141,4 +142,50 @@ def test_c5_sampled(T):
     toks = W.sample_tokens(sh, inp["topk_ids"], 48)
     got = gpu_forward(sh, inp)
     ref = oracle_forward(sh, inp, tokens=toks)
-    check(sh, got[toks], ref[toks], f"C5 T={T}")
+    rel, cos = check(sh, got[toks], ref[toks], f"C5 T={T}")
+    print(f"PARITY C5 T={T} tokens={len(toks)} max|diff|/rms={rel:.3e} cos={cos:.7f}")
+
+
+# ---------------------------------------------------------------- full-size workloads, sampled tokens
+_WEIGHTS = {}
+
+
+def _weights(name):
+    """Expert weights of a named workload, generated once per test session."""
+    if name not in _WEIGHTS:
+        _WEIGHTS.clear()  # hold one workload's weights at a time (C4 is ~26 GB in mxfp8)
+        sh = W.shape(name)
+        if sh.dtype == "bf16":
+            _WEIGHTS[name] = dict(w1=W.bf16_weights(sh, "w1"), w2=W.bf16_weights(sh, "w2"))
+        else:
+            w1, s1 = W.mxfp8_weights(sh, "w1")
+            w2, s2 = W.mxfp8_weights(sh, "w2")
+            _WEIGHTS[name] = dict(w1=w1, w1_scales=s1, w2=w2, w2_scales=s2)
+    return _WEIGHTS[name]
+
+
+def _full_inputs(name, T):
+    sh = W.shape(name, T)
+    ids, tw = W.routing(sh)
+    inp = dict(_weights(name), topk_ids=ids, topk_weights=tw)
+    if sh.dtype == "bf16":
+        inp["x"] = W.f32_to_bf16_bits(W.x_f32(sh))
+    else:
+        inp["x"], inp["x_scales"] = W.mx_quantize_inputs(W.x_f32(sh))
+    return sh, inp
+
+
+@pytest.mark.parametrize("name,T,ntok", [("C2", 64, 32), ("C2", 256, 32),
+                                         ("C3", 64, 12), ("C3", 256, 12), ("C3", 1024, 12), ("C3", 2048, 12),
+                                         ("C3", 4096, 12), ("C3", 8192, 12),
+                                         ("C4", 1024, 6), ("C4", 2048, 6), ("C4", 4096, 6), ("C4", 8192, 6)])
+def test_full_size_sampled(name, T, ntok):
+    """The workload at full size through the GPU path; parity on a seeded token
+    sample that includes tokens of the most- and least-loaded experts."""
+    sh, inp = _full_inputs(name, T)
+    toks = W.sample_tokens(sh, inp["topk_ids"], ntok)
+    got = gpu_forward(sh, inp)
+    ref = oracle_forward(sh, inp, tokens=toks)
+    rel, cos = check(sh, got[toks], ref[toks], f"{name} T={T}")
+    assert np.isfinite(W.bf16_bits_to_f32(got)).all()
+    print(f"PARITY {name} T={T} tokens={len(toks)} max|diff|/rms={rel:.3e} cos={cos:.7f}")
