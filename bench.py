@@ -287,7 +287,9 @@ class Problem:
             m.fused_moe_mxfp8(self.x, self.xs, self.w1, self.s1, self.w2, self.s2, self.s_ids, self.e_ids, self.ntpp,
                               self.tw, self.out, self.bm, workspace=self.ws, tune=tune)
 
-    def step(self, tune=None):
+    def step(self, tune=None, plan_event=None):
+        if plan_event is not None:
+            plan_event.record()
         self.moe.moe_align(self.ids, self.sh.E, self.bm, self.s_ids, self.e_ids, self.ntpp)
         self.fused(self.plain if tune is None else tune)
 
@@ -303,6 +305,7 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
     moe = prob.moe
     stream = torch.cuda.current_stream()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    pev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     tunes = [moe.Tuning.with_events(e, prob.stages, prob.ctas) for e in ev]
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=prob.dev) if flush_l2 else None
     for _ in range(max(3, warmup)):
@@ -324,7 +327,7 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
     for i in range(steps):
         if s_ev:
             s_ev[i][0].record(stream)
-        prob.step(tunes[i])
+        prob.step(tunes[i], pev[i])
         if s_ev:
             s_ev[i][1].record(stream)
             flush.fill_(1)
@@ -339,6 +342,7 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
     else:
         total_ms = t0.elapsed_time(t1)
     return {"total_ms": total_ms, "ms_step": total_ms / steps,
+            "plan_ms": sum(a.elapsed_time(e[0]) for a, e in zip(pev, ev)) / steps,
             "p1_ms": sum(e[0].elapsed_time(e[1]) for e in ev) / steps,
             "p2_ms": sum(e[1].elapsed_time(e[2]) for e in ev) / steps,
             "cb_ms": sum(e[2].elapsed_time(e[3]) for e in ev) / steps,
@@ -420,7 +424,8 @@ def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
                           "frac": cm["t_roof"] / (ms_step * 1e-3), "touched_experts": cm["touched"],
                           "routed_gflop": cm["flops"] / 1e9, "touched_weight_gb": cm["bytes_w"] / 1e9,
                           "peaks": peak_src},
-        "phase_us": {"gate_up": m["p1_ms"] * 1e3, "down": m["p2_ms"] * 1e3, "reduce": m["cb_ms"] * 1e3},
+        "phase_us": {"planner": m["plan_ms"] * 1e3, "gate_up": m["p1_ms"] * 1e3, "down": m["p2_ms"] * 1e3,
+                     "reduce": m["cb_ms"] * 1e3},
         "roofline": roofline_of_p1(sh, cm, m["p1_ms"], peaks, peak_src),
         "gpu_launches": m["launches"],
         "clocks": m["clocks"],

@@ -28,7 +28,9 @@
 //   phase 2  persistent kernel, unit = (block b, 256 output features).  A =
 //            the block's intermediate rows (TMA), B = 256 rows of w2[e] (TMA),
 //            D in TMEM; each epilogue thread scales its row by the routing
-//            weight and writes one fp32 row segment per route.
+//            weight and writes one row segment per route (fp32 on the bf16
+//            path; bf16 on the mxfp8 path, whose tolerance leaves room for
+//            the extra rounding).
 //   combine  out[t] = bf16(sum over the token's routes, in route order), a
 //            deterministic HBM-bound pass.
 // The weight tiles are streamed once per unit through a multi-stage shared
@@ -97,7 +99,7 @@ struct P2Params {
   const int32_t* expert_ids;
   const int32_t* ntpp;
   const float* topk_w;
-  float* yw;                // (R, K) weighted down-projection rows
+  void* yw;                 // (R, K) weighted down-projection rows: fp32 (bf16 path) or bf16 (mxfp8 path)
   int32_t* flags;
   int* status;
   int K, I, E, top_k, bm, R;
@@ -601,7 +603,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     const int q = warp & 3;
     const int h = (warp - kP2FirstEpi) >> 2;
     const int r = 32 * q + lane;
-    float4* stg4 = reinterpret_cast<float4*>(ctrl + kP2Ctrl) + (warp - kP2FirstEpi) * (kStageFloatsPerWarp / 4);
+    uint4* stg4 = reinterpret_cast<uint4*>(ctrl + kP2Ctrl) + (warp - kP2FirstEpi) * (kStageFloatsPerWarp / 4);
     int acc_it = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -626,10 +628,14 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       tc_fence_after();
       const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 256u;
       if (32 * q < bi.nend) {
-        // Thread = row.  Each 16-column slice of the warp's 32 rows goes
-        // through shared memory so that the stores leave as 64 contiguous
-        // bytes per row (8 rows per instruction) instead of 16 bytes to 32
-        // different rows.  float4 slot i of row l sits at i ^ (l & 3).
+        // Thread = row.  Each slice of the warp's 32 rows goes through shared
+        // memory so that the stores leave as 64 contiguous bytes per row (8
+        // rows per instruction) instead of 16 bytes to 32 different rows.
+        // 16-byte slot i of row l sits at i ^ ((l >> 1) & 3), so both the
+        // row-per-lane writes and the 8-rows-per-instruction reads touch all
+        // 32 banks (4 wavefronts per 512 bytes).  The bf16 path keeps the
+        // weighted rows in fp32 (16 columns per slice); the mxfp8 path rounds
+        // them to bf16 (32 columns per slice), half the bytes.
         const int half = nn / 2;
         const int64_t col_base = static_cast<int64_t>(ht) * kTH + h * half;
 #pragma unroll 1
@@ -638,25 +644,40 @@ __global__ void __launch_bounds__(kP2Threads, 1)
           tmem_ld32(tacc + h * half + c, yr);
           tmem_ld_wait();
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
+          for (int hh = 0; hh < (kFp8 ? 1 : 2); ++hh) {
             __syncwarp();
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const int k = 16 * hh + 4 * i;
-              stg4[lane * 4 + (i ^ (lane & 3))] =
-                  make_float4(wgt * __uint_as_float(yr[k]), wgt * __uint_as_float(yr[k + 1]),
-                              wgt * __uint_as_float(yr[k + 2]), wgt * __uint_as_float(yr[k + 3]));
+              uint4 w;
+              if (kFp8) {
+                const int k = 8 * i;
+                w = make_uint4(pack_bf16x2(wgt * __uint_as_float(yr[k]), wgt * __uint_as_float(yr[k + 1])),
+                               pack_bf16x2(wgt * __uint_as_float(yr[k + 2]), wgt * __uint_as_float(yr[k + 3])),
+                               pack_bf16x2(wgt * __uint_as_float(yr[k + 4]), wgt * __uint_as_float(yr[k + 5])),
+                               pack_bf16x2(wgt * __uint_as_float(yr[k + 6]), wgt * __uint_as_float(yr[k + 7])));
+              } else {
+                const int k = 16 * hh + 4 * i;
+                w = make_uint4(__float_as_uint(wgt * __uint_as_float(yr[k])),
+                               __float_as_uint(wgt * __uint_as_float(yr[k + 1])),
+                               __float_as_uint(wgt * __uint_as_float(yr[k + 2])),
+                               __float_as_uint(wgt * __uint_as_float(yr[k + 3])));
+              }
+              stg4[lane * 4 + (i ^ ((lane >> 1) & 3))] = w;
             }
             __syncwarp();
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
               const int rl = 8 * it + (lane >> 2), cq = lane & 3;
-              const float4 v = stg4[rl * 4 + (cq ^ (rl & 3))];
+              const uint4 v = stg4[rl * 4 + (cq ^ ((rl >> 1) & 3))];
               const int route_l = __shfl_sync(0xffffffffu, route, rl);
               const int mine_l = __shfl_sync(0xffffffffu, static_cast<int>(mine), rl);
-              if (mine_l)
-                *reinterpret_cast<float4*>(p.yw + static_cast<int64_t>(route_l) * p.K + col_base + c + 16 * hh +
-                                           4 * cq) = v;
+              if (mine_l) {
+                const int64_t e0 = static_cast<int64_t>(route_l) * p.K + col_base + c;
+                if (kFp8)
+                  *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.yw) + e0 + 8 * cq) = v;
+                else
+                  *reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.yw) + e0 + 16 * hh + 4 * cq) = v;
+              }
             }
           }
         }
@@ -681,7 +702,22 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 // ========================================================================
 // combine: out[t] = bf16( sum_j yw[t*top_k + j] ), routes in order
 // ========================================================================
-__global__ void moe_combine_kernel(const float* __restrict__ yw, const int32_t* __restrict__ flags,
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+template <typename TP>
+__global__ void moe_combine_kernel(const TP* __restrict__ yw, const int32_t* __restrict__ flags,
                                    __nv_bfloat16* __restrict__ out, int T, int K, int top_k) {
   const int kv = K / 8;
   const int64_t n = static_cast<int64_t>(T) * kv;
@@ -693,10 +729,10 @@ __global__ void moe_combine_kernel(const float* __restrict__ yw, const int32_t* 
     for (int j = 0; j < top_k; ++j) {
       const int64_t r = t * top_k + j;
       if (__ldg(flags + r)) {
-        const float4* src = reinterpret_cast<const float4*>(yw + r * K + h);
-        const float4 a = __ldg(src), bb = __ldg(src + 1);
-        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-        acc[4] += bb.x; acc[5] += bb.y; acc[6] += bb.z; acc[7] += bb.w;
+        float y[8];
+        load8(yw + r * K + h, y);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += y[i];
       }
     }
     __nv_bfloat162 o[4];
@@ -728,7 +764,7 @@ static WsLayout ws_layout(bool fp8, int T, int K, int N, int E, int top_k, int b
   w.act_sf = off;
   if (fp8) off = round_up(off + (w.cap_rows / bm) * (I / 128) * kSfTileBytes, 1024);
   w.yw = off;
-  off = round_up(off + R * K * 4, 1024);
+  off = round_up(off + R * K * (fp8 ? 2 : 4), 1024);
   w.flags = off;
   off = round_up(off + R * 4, 256);
   w.total = off;
@@ -899,7 +935,7 @@ static int run_fused(const FusedArgs& a) {
   p2.expert_ids = a.expert_ids;
   p2.ntpp = a.ntpp;
   p2.topk_w = a.topk_w;
-  p2.yw = reinterpret_cast<float*>(ws + L.yw);
+  p2.yw = ws + L.yw;
   p2.flags = p1.flags;
   p2.status = p1.status;
   p2.K = a.K; p2.I = I; p2.E = a.E; p2.top_k = a.top_k; p2.bm = a.bm; p2.R = p1.R;
@@ -947,9 +983,14 @@ static int run_fused(const FusedArgs& a) {
   if ((rc = mark(2)) != MOE_OK) return rc;
   const int64_t nvec = static_cast<int64_t>(a.T) * (a.K / 8);
   const int64_t cblocks = (nvec + 255) / 256;
-  moe_combine_kernel<<<static_cast<int>(cblocks < 4L * nsm ? cblocks : 4L * nsm), 256, 0, a.stream>>>(
-      reinterpret_cast<const float*>(ws + L.yw), p1.flags, static_cast<__nv_bfloat16*>(a.out), a.T, a.K,
-      a.top_k);
+  const int cgrid = static_cast<int>(cblocks < 4L * nsm ? cblocks : 4L * nsm);
+  if (a.fp8)
+    moe_combine_kernel<__nv_bfloat16><<<cgrid, 256, 0, a.stream>>>(
+        reinterpret_cast<const __nv_bfloat16*>(ws + L.yw), p1.flags, static_cast<__nv_bfloat16*>(a.out), a.T, a.K,
+        a.top_k);
+  else
+    moe_combine_kernel<float><<<cgrid, 256, 0, a.stream>>>(reinterpret_cast<const float*>(ws + L.yw), p1.flags,
+                                                           static_cast<__nv_bfloat16*>(a.out), a.T, a.K, a.top_k);
   err = cudaGetLastError();
   if (err != cudaSuccess) return cuda_fail("fused_moe: combine launch", err);
   return mark(3);

@@ -10,7 +10,10 @@
 // num_tokens_post_padded is the padded total.
 //
 // One CTA of 32 warps does the three phases in shared memory, so no grid-wide
-// synchronisation is needed:
+// synchronisation is needed.  When they fit (uint16 each, next to the
+// histograms), the R expert ids are first staged in shared memory with
+// independent loads, so the two passes below read shared memory instead of
+// waiting on one global load per 32 ids:
 //   1. warp w owns the contiguous id range [w*chunk, (w+1)*chunk) and counts
 //      it into its private histogram row hist[w][:] (lanes with the same
 //      expert are grouped with __match_any_sync; the group leader adds the
@@ -29,20 +32,46 @@ namespace moe {
 
 constexpr int kAlignThreads = 1024;
 constexpr int kAlignWarps = kAlignThreads / 32;
+constexpr int kAlignSmemLimit = 232448;
+constexpr uint16_t kNoExpert = 0xFFFFu;
+
+// Shared memory: hist[kAlignWarps][E], count[E], off[E + 1], warp_tot[kAlignWarps]
+// (int32), then -- when they fit -- the R expert ids as uint16.
+__host__ __device__ inline size_t align_smem_base(int E) {
+  return sizeof(int32_t) * (static_cast<size_t>(kAlignWarps) * E + E + E + 1 + kAlignWarps);
+}
 
 __global__ void __launch_bounds__(kAlignThreads, 1)
     moe_align_kernel(const int32_t* __restrict__ topk_ids, int R, int E, int block_m,
                      int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids,
-                     int32_t* __restrict__ ntpp_out, int64_t capacity) {
+                     int32_t* __restrict__ ntpp_out, int64_t capacity, int staged) {
   extern __shared__ int32_t sm[];
   int32_t* hist = sm;                         // [kAlignWarps][E], later start offsets
   int32_t* count = hist + kAlignWarps * E;    // [E]
   int32_t* off = count + E;                   // [E + 1]
   int32_t* warp_tot = off + E + 1;            // [kAlignWarps]
+  uint16_t* ids16 = reinterpret_cast<uint16_t*>(warp_tot + kAlignWarps);  // [R] when staged
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < kAlignWarps * E; i += kAlignThreads) hist[i] = 0;
+  // 0. stage the ids (independent loads, so their latencies overlap); ids
+  //    outside [0, E) route nowhere
+  if (staged) {
+#pragma unroll 4
+    for (int i = tid; i < R; i += kAlignThreads) {
+      const int e = __ldg(topk_ids + i);
+      ids16[i] = (e >= 0 && e < E) ? static_cast<uint16_t>(e) : kNoExpert;
+    }
+  }
   __syncthreads();
+  auto expert_of = [&](int i) -> int {
+    if (staged) {
+      const uint16_t v = ids16[i];
+      return v == kNoExpert ? -1 : static_cast<int>(v);
+    }
+    const int e = __ldg(topk_ids + i);
+    return (e >= 0 && e < E) ? e : -1;
+  };
 
   const int chunk = (R + kAlignWarps - 1) / kAlignWarps;
   const int lo = min(R, warp * chunk), hi = min(R, lo + chunk);
@@ -51,8 +80,7 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
   // 1. warp-private histograms
   for (int base = lo; base < hi; base += 32) {
     const int i = base + lane;
-    int e = (i < hi) ? topk_ids[i] : -1;
-    if (e >= E) e = -1;
+    const int e = (i < hi) ? expert_of(i) : -1;
     const unsigned same = __match_any_sync(0xffffffffu, e);
     if (e >= 0 && (same & lt_mask) == 0) hist[warp * E + e] += __popc(same);
     __syncwarp();
@@ -109,8 +137,7 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
   // 3. stable scatter
   for (int base = lo; base < hi; base += 32) {
     const int i = base + lane;
-    int e = (i < hi) ? topk_ids[i] : -1;
-    if (e >= E) e = -1;
+    const int e = (i < hi) ? expert_of(i) : -1;
     const unsigned same = __match_any_sync(0xffffffffu, e);
     if (e >= 0) {
       const int rank = __popc(same & lt_mask);
@@ -159,19 +186,22 @@ extern "C" int moe_align(const int32_t* topk_ids, int T, int top_k, int E, int b
   if ((T > 0 && !topk_ids) || !sorted_token_ids || !expert_ids || !num_tokens_post_padded)
     return fail(MOE_ERR_INVALID_ARG, "moe_align: null pointer");
 
-  const size_t smem = sizeof(int32_t) * (static_cast<size_t>(kAlignWarps) * E + E + E + 1 + kAlignWarps);
+  const int R = T * top_k;
+  const size_t base = align_smem_base(E);
+  const size_t staged_bytes = base + sizeof(uint16_t) * static_cast<size_t>(R);
+  const int staged = staged_bytes <= static_cast<size_t>(kAlignSmemLimit) ? 1 : 0;
+  const size_t smem = staged ? staged_bytes : base;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("moe_align: cudaGetDevice");
   static bool attr_set[kMaxDevices] = {};
   if (dev < kMaxDevices && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(moe_align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(sizeof(int32_t) * (kAlignWarps * kMaxExperts + 2 * kMaxExperts +
-                                                                 1 + kAlignWarps))) != cudaSuccess)
+    if (cudaFuncSetAttribute(moe_align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAlignSmemLimit) !=
+        cudaSuccess)
       return cuda_fail("moe_align: cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
   moe_align_kernel<<<1, kAlignThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
-      topk_ids, T * top_k, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded, capacity);
+      topk_ids, R, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded, capacity, staged);
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return cuda_fail("moe_align: launch", err);
   return MOE_OK;
