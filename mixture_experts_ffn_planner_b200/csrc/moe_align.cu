@@ -9,23 +9,29 @@
 // padded to block_m with -1; expert_ids names the expert of each block;
 // num_tokens_post_padded is the padded total.
 //
-// One CTA of 32 warps does the three phases in shared memory, so no grid-wide
-// synchronisation is needed.  When they fit (uint16 each, next to the
-// histograms), the R expert ids are first staged in shared memory with
-// independent loads, so the two passes below read shared memory instead of
-// waiting on one global load per 32 ids:
-//   1. warp w owns the contiguous id range [w*chunk, (w+1)*chunk) and counts
-//      it into its private histogram row hist[w][:] (lanes with the same
-//      expert are grouped with __match_any_sync; the group leader adds the
-//      group size -- no atomics);
-//   2. per expert, the rows are scanned over w (giving each warp its start
-//      inside the expert's segment) and the padded counts are scanned over e
-//      (the segment offsets);
+// The planner runs as one thread-block cluster of C CTAs (C = 1 for small
+// inputs, 8 otherwise) of 32 warps; the CTAs exchange their per-expert counts
+// through distributed shared memory, so neither global scratch nor a
+// grid-wide synchronisation is needed.  CTA c owns the contiguous id range
+// [c*chunk, (c+1)*chunk) and, inside it, warp w a contiguous sub-range:
+//   0. the CTA's ids are staged in shared memory as uint16 with independent
+//      loads (when they fit; otherwise they are re-read from global memory);
+//   1. every warp counts its sub-range into a private histogram row
+//      hist[w][:] (lanes with the same expert are grouped with
+//      __match_any_sync; the group leader adds the group size -- no atomics);
+//      per expert the rows are then scanned over w, giving each warp its start
+//      inside the CTA's share, and the CTA total cnt[e] is published;
+//   2. after a cluster barrier every CTA reads all CTAs' cnt[e] through
+//      distributed shared memory: before[e] (the counts of lower CTAs) and
+//      the expert totals, whose padded exclusive scan gives the segment
+//      offsets off[e] (computed identically in every CTA);
 //   3. every warp walks its range again and writes each id to
-//      off[e] + start[w][e] + (rank among earlier lanes with the same expert),
-//      so ids ascend inside a segment -- the result is unique and bit-exact.
+//      off[e] + before[e] + start[w][e] + (rank among earlier lanes with the
+//      same expert), so ids ascend inside a segment -- the result is unique
+//      and bit-exact.
 // Slots that receive no id (segment padding and the capacity tail) get -1,
-// and expert_ids is filled block by block.
+// and expert_ids is filled block by block; these writes are spread over the
+// cluster's CTAs.
 #include "internal.h"
 
 namespace moe {
@@ -33,12 +39,37 @@ namespace moe {
 constexpr int kAlignThreads = 1024;
 constexpr int kAlignWarps = kAlignThreads / 32;
 constexpr int kAlignSmemLimit = 232448;
+constexpr int kAlignClusterMax = 8;
+constexpr int kAlignClusterMinIds = 4096;  // inputs smaller than this use one CTA
 constexpr uint16_t kNoExpert = 0xFFFFu;
 
-// Shared memory: hist[kAlignWarps][E], count[E], off[E + 1], warp_tot[kAlignWarps]
-// (int32), then -- when they fit -- the R expert ids as uint16.
+// Shared memory (int32): hist[kAlignWarps][E], cnt[E], before[E], off[E + 1],
+// warp_tot[kAlignWarps]; then -- when they fit -- the CTA's ids as uint16.
 __host__ __device__ inline size_t align_smem_base(int E) {
-  return sizeof(int32_t) * (static_cast<size_t>(kAlignWarps) * E + E + E + 1 + kAlignWarps);
+  return sizeof(int32_t) * (static_cast<size_t>(kAlignWarps) * E + 3 * static_cast<size_t>(E) + 1 + kAlignWarps);
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Reads a 32-bit word of CTA `rank`'s shared memory at the address that
+// `local` has in this CTA.
+__device__ __forceinline__ int32_t ld_dsmem(const int32_t* local, uint32_t rank) {
+  uint32_t remote;
+  int32_t v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(local))), "r"(rank));
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
+  return v;
 }
 
 __global__ void __launch_bounds__(kAlignThreads, 1)
@@ -47,37 +78,42 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
                      int32_t* __restrict__ ntpp_out, int64_t capacity, int staged) {
   extern __shared__ int32_t sm[];
   int32_t* hist = sm;                         // [kAlignWarps][E], later start offsets
-  int32_t* count = hist + kAlignWarps * E;    // [E]
-  int32_t* off = count + E;                   // [E + 1]
+  int32_t* cnt = hist + kAlignWarps * E;      // [E] this CTA's count per expert
+  int32_t* before = cnt + E;                  // [E] counts of lower-ranked CTAs
+  int32_t* off = before + E;                  // [E + 1] segment offsets
   int32_t* warp_tot = off + E + 1;            // [kAlignWarps]
-  uint16_t* ids16 = reinterpret_cast<uint16_t*>(warp_tot + kAlignWarps);  // [R] when staged
+  uint16_t* ids16 = reinterpret_cast<uint16_t*>(warp_tot + kAlignWarps);  // [chunk] when staged
 
+  const uint32_t crank = cluster_ctarank(), csize = cluster_nctarank();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cchunk = (R + static_cast<int>(csize) - 1) / static_cast<int>(csize);
+  const int clo = min(R, static_cast<int>(crank) * cchunk), chi = min(R, clo + cchunk);
+
   for (int i = tid; i < kAlignWarps * E; i += kAlignThreads) hist[i] = 0;
-  // 0. stage the ids (independent loads, so their latencies overlap); ids
-  //    outside [0, E) route nowhere
+  // 0. stage this CTA's ids (independent loads, so their latencies overlap);
+  //    ids outside [0, E) route nowhere
   if (staged) {
 #pragma unroll 4
-    for (int i = tid; i < R; i += kAlignThreads) {
+    for (int i = clo + tid; i < chi; i += kAlignThreads) {
       const int e = __ldg(topk_ids + i);
-      ids16[i] = (e >= 0 && e < E) ? static_cast<uint16_t>(e) : kNoExpert;
+      ids16[i - clo] = (e >= 0 && e < E) ? static_cast<uint16_t>(e) : kNoExpert;
     }
   }
   __syncthreads();
   auto expert_of = [&](int i) -> int {
     if (staged) {
-      const uint16_t v = ids16[i];
+      const uint16_t v = ids16[i - clo];
       return v == kNoExpert ? -1 : static_cast<int>(v);
     }
     const int e = __ldg(topk_ids + i);
     return (e >= 0 && e < E) ? e : -1;
   };
 
-  const int chunk = (R + kAlignWarps - 1) / kAlignWarps;
-  const int lo = min(R, warp * chunk), hi = min(R, lo + chunk);
+  const int wchunk = (chi - clo + kAlignWarps - 1) / kAlignWarps;
+  const int lo = min(chi, clo + warp * wchunk), hi = min(chi, lo + wchunk);
   const unsigned lt_mask = (1u << lane) - 1u;
 
-  // 1. warp-private histograms
+  // 1. warp-private histograms, then the scan over warps and the CTA count
   for (int base = lo; base < hi; base += 32) {
     const int i = base + lane;
     const int e = (i < hi) ? expert_of(i) : -1;
@@ -86,8 +122,6 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     __syncwarp();
   }
   __syncthreads();
-
-  // 2a. per expert: exclusive scan over warps, total count
   for (int e = tid; e < E; e += kAlignThreads) {
     int run = 0;
     for (int w = 0; w < kAlignWarps; ++w) {
@@ -95,16 +129,30 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
       hist[w * E + e] = run;
       run += c;
     }
-    count[e] = run;
+    cnt[e] = run;
   }
-  __syncthreads();
+  cluster_sync();  // every CTA's cnt[] is published
 
-  // 2b. exclusive scan of the padded counts over experts (block-wide, in
-  // rounds of kAlignThreads experts)
+  // 2a. counts of lower CTAs and expert totals, read from every CTA; the
+  //     totals are parked in off[] until the scan replaces them
+  for (int e = tid; e < E; e += kAlignThreads) {
+    int lower = 0, total = 0;
+    for (uint32_t c = 0; c < csize; ++c) {
+      const int v = (c == crank) ? cnt[e] : ld_dsmem(cnt + e, c);
+      if (c < crank) lower += v;
+      total += v;
+    }
+    before[e] = lower;
+    off[e] = total;  // total for now; replaced by the offset below
+  }
+  cluster_sync();  // no CTA reads another's shared memory after this point
+
+  // 2b. exclusive scan of the padded totals over experts (block-wide, in
+  // rounds of kAlignThreads experts); identical in every CTA
   int carry = 0;
   for (int e0 = 0; e0 < E; e0 += kAlignThreads) {
     const int e = e0 + tid;
-    const int padded = (e < E) ? (count[e] + block_m - 1) / block_m * block_m : 0;
+    const int padded = (e < E) ? (off[e] + block_m - 1) / block_m * block_m : 0;
     int v = padded;
     for (int d = 1; d < 32; d <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, v, d);
@@ -122,14 +170,19 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     }
     __syncthreads();
     const int incl = v + (warp > 0 ? warp_tot[warp - 1] : 0) + carry;
-    if (e < E) off[e] = incl - padded;
+    const int total = (e < E) ? off[e] : 0;
+    __syncthreads();
+    if (e < E) {
+      off[e] = incl - padded;
+      cnt[e] = total;  // cnt now holds the expert total
+    }
     const int round_total = warp_tot[kAlignWarps - 1];
     __syncthreads();
     carry += round_total;
   }
   if (tid == 0) {
     off[E] = carry;
-    *ntpp_out = carry;
+    if (crank == 0) *ntpp_out = carry;
   }
   __syncthreads();
   const int ntpp = off[E];
@@ -141,22 +194,25 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
     const unsigned same = __match_any_sync(0xffffffffu, e);
     if (e >= 0) {
       const int rank = __popc(same & lt_mask);
-      sorted_ids[off[e] + hist[warp * E + e] + rank] = i;
+      sorted_ids[off[e] + before[e] + hist[warp * E + e] + rank] = i;
     }
     __syncwarp();
     if (e >= 0 && (same & lt_mask) == 0) hist[warp * E + e] += __popc(same);
     __syncwarp();
   }
 
-  // padding inside each segment, then the capacity tail
-  for (int e = warp; e < E; e += kAlignWarps) {
-    const int s = off[e] + count[e], t = off[e + 1];
+  // padding inside each segment (expert e by CTA e % csize), then the
+  // capacity tail (strided over the cluster)
+  for (int e = static_cast<int>(crank) * kAlignWarps + warp; e < E; e += static_cast<int>(csize) * kAlignWarps) {
+    const int s = off[e] + cnt[e], t = off[e + 1];
     for (int p = s + lane; p < t; p += 32) sorted_ids[p] = -1;
     for (int b = off[e] / block_m + lane; b < t / block_m; b += 32) expert_ids[b] = e;
   }
-  for (int64_t p = ntpp + tid; p < capacity; p += kAlignThreads) sorted_ids[p] = -1;
+  const int64_t stride = static_cast<int64_t>(csize) * kAlignThreads;
+  const int64_t first = static_cast<int64_t>(crank) * kAlignThreads + tid;
+  for (int64_t p = ntpp + first; p < capacity; p += stride) sorted_ids[p] = -1;
   const int64_t nblk_cap = (capacity + block_m - 1) / block_m;
-  for (int64_t b = ntpp / block_m + tid; b < nblk_cap; b += kAlignThreads) expert_ids[b] = -1;
+  for (int64_t b = ntpp / block_m + first; b < nblk_cap; b += stride) expert_ids[b] = -1;
 }
 
 }  // namespace moe
@@ -187,8 +243,10 @@ extern "C" int moe_align(const int32_t* topk_ids, int T, int top_k, int E, int b
     return fail(MOE_ERR_INVALID_ARG, "moe_align: null pointer");
 
   const int R = T * top_k;
+  const int csize = R >= kAlignClusterMinIds ? kAlignClusterMax : 1;
+  const int cchunk = (R + csize - 1) / csize;
   const size_t base = align_smem_base(E);
-  const size_t staged_bytes = base + sizeof(uint16_t) * static_cast<size_t>(R);
+  const size_t staged_bytes = base + sizeof(uint16_t) * static_cast<size_t>(cchunk);
   const int staged = staged_bytes <= static_cast<size_t>(kAlignSmemLimit) ? 1 : 0;
   const size_t smem = staged ? staged_bytes : base;
   int dev = 0;
@@ -200,8 +258,21 @@ extern "C" int moe_align(const int32_t* topk_ids, int T, int top_k, int E, int b
       return cuda_fail("moe_align: cudaFuncSetAttribute");
     attr_set[dev] = true;
   }
-  moe_align_kernel<<<1, kAlignThreads, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
-      topk_ids, R, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded, capacity, staged);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(csize, 1, 1);
+  cfg.blockDim = dim3(kAlignThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t lerr = cudaLaunchKernelEx(&cfg, moe_align_kernel, topk_ids, R, E, block_m, sorted_token_ids,
+                                              expert_ids, num_tokens_post_padded, capacity, staged);
+  if (lerr != cudaSuccess) return cuda_fail("moe_align: launch", lerr);
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return cuda_fail("moe_align: launch", err);
   return MOE_OK;

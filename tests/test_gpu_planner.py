@@ -45,7 +45,7 @@ def _check(ids, E, bm, cap=None):
 @pytest.mark.parametrize("bm", [16, 32, 64, 128])
 @pytest.mark.parametrize("T,k,E", [(1, 1, 1), (7, 2, 4), (100, 3, 9), (333, 8, 64), (2048, 6, 256),
                                    (5000, 4, 1024), (4097, 8, 288),
-                                   (12000, 4, 1024)])  # ids too many to stage in shared memory: streaming path
+                                   (12000, 4, 1024), (90000, 4, 1024)])  # the last: ids streamed, not staged
 def test_random(T, k, E, bm):
     rng = np.random.default_rng(T * 131 + k * 7 + E + bm)
     ids = np.stack([rng.permutation(E)[:k] if k <= E else rng.integers(0, E, k) for _ in range(T)]).astype(np.int32)
