@@ -46,8 +46,8 @@ namespace moe {
 __device__ int g_moe_status = 0;
 
 constexpr int kM = 128;           // MMA M: routed rows of one planner block (rows >= block_m unused)
-constexpr int kTI = 128;          // intermediate columns per phase-1 unit (gate 128 + up 128 = MMA N 256)
-constexpr int kTH = 256;          // output features per phase-2 unit (MMA N)
+constexpr int kTI = 128;          // intermediate columns per gate/up unit (gate 128 + up 128 = MMA N 256)
+constexpr int kTH = 256;          // output features per down unit (MMA N)
 constexpr int kRowBytes = 128;    // bytes of one operand row per pipeline stage
 constexpr int kSfTileBytes = 512; // one blocked scale tile: 128 rows x 4 scales
 constexpr int kSmemLimit = 232448;  // 227 KB of dynamic shared memory per CTA
@@ -88,7 +88,7 @@ struct P1Params {
   int* status;
   int K, N, I, E, top_k, bm, R;
   int max_blocks;           // blocks a kernel may visit
-  int n_jt;                 // ceil(I / 128)
+  int n_jt;                 // ceil(I / 128): work units per planner block
   int stages, stage_bytes;
 };
 
@@ -104,7 +104,7 @@ struct P2Params {
   int* status;
   int K, I, E, top_k, bm, R;
   int max_blocks;
-  int n_ht;                 // ceil(K / 256)
+  int n_ht;                 // ceil(K / 256): work units per planner block
   int n_kc;                 // K-chunks of the down GEMM
   int stages, stage_bytes;
 };
@@ -137,6 +137,55 @@ __device__ __forceinline__ BlockInfo block_info(const int32_t* sorted_ids, const
   if (bi.e < 0 || bi.e >= E) bi.nend = 0;
   bi.n16 = (bi.nend + 15) & ~15;
   return bi;
+}
+
+// The global reads block_info needs, issued one unit ahead: every role
+// prefetches the next unit's expert id and row ids into registers while it
+// works on the current unit, so the loads' latency never sits on the
+// pipeline's critical path.  Lane l holds rows l, l+32, l+64, l+96.
+struct BlockPf {
+  int e;
+  int id[4];
+};
+
+__device__ __forceinline__ BlockPf block_prefetch(const int32_t* sorted_ids, const int32_t* expert_ids, int u,
+                                                  int n_units, int per_block, int bm) {
+  BlockPf f;
+  f.e = -1;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) f.id[q] = -1;
+  if (u < n_units) {
+    const int b = u / per_block;
+    const int lane = static_cast<int>(lane_id());
+    f.e = __ldg(expert_ids + b);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int r = 32 * q + lane;
+      if (r < bm) f.id[q] = __ldg(sorted_ids + static_cast<int64_t>(b) * bm + r);
+    }
+  }
+  return f;
+}
+
+// block_info from prefetched data (warp-collective).
+__device__ __forceinline__ BlockInfo block_finalize(const BlockPf& f, int R, int E) {
+  BlockInfo bi;
+  bi.e = f.e;
+  bi.nend = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const bool v = f.id[q] >= 0 && f.id[q] < R;
+    bi.vm[q] = __ballot_sync(0xffffffffu, v);
+    if (bi.vm[q]) bi.nend = 32 * q + 32 - __clz(static_cast<int>(bi.vm[q]));
+  }
+  if (bi.e < 0 || bi.e >= E) bi.nend = 0;
+  bi.n16 = (bi.nend + 15) & ~15;
+  return bi;
+}
+
+// f.id[q] for a warp-uniform or per-thread q in 0..3 without local memory.
+__device__ __forceinline__ int pf_id(const BlockPf& f, int q) {
+  return q == 0 ? f.id[0] : q == 1 ? f.id[1] : q == 2 ? f.id[2] : f.id[3];
 }
 
 __device__ __forceinline__ bool row_valid(const BlockInfo& bi, int c) {
@@ -214,7 +263,8 @@ __global__ void __launch_bounds__(kP1Threads, 1)
   const uint32_t tbase = *tmem_base_sm;
 
   const int n_blocks = num_blocks(p.ntpp, p.bm, p.max_blocks);
-  const int n_units = n_blocks * p.n_jt;
+  const int n_jt = p.n_jt;
+  const int n_units = n_blocks * n_jt;
   constexpr int kKC = kFp8 ? 128 : 64;  // K elements per stage (128 bytes per row)
   const int n_kc = p.K / kKC;
   const int esize = kFp8 ? 1 : 2;
@@ -224,14 +274,17 @@ __global__ void __launch_bounds__(kP1Threads, 1)
   if (warp == 0) {
     // ------------------------------------------------ TMA producer (weights)
     const uint64_t pol = policy_evict_first();
-    const uint32_t tx = 2 * 128 * kRowBytes + (kFp8 ? 2 * kSfTileBytes : 0);
+    const uint32_t tx = 2 * kTI * kRowBytes + (kFp8 ? 2 * kSfTileBytes : 0);
     const int MT1 = p.N / 128, KT1 = p.K / 128;
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_jt, p.bm);
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int b = u / p.n_jt, j = u - (u / p.n_jt) * p.n_jt;
-      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      const int j = u - (u / n_jt) * n_jt;
+      const BlockPf cur = pf;
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_jt, p.bm);
+      const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
       const int gate_row = bi.e * p.N + j * kTI;
       const int up_row = bi.e * p.N + p.I + j * kTI;
@@ -264,9 +317,11 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     uint32_t ph = 0;
     int acc_it = 0;
     bool ok = true;
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_jt, p.bm);
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int b = u / p.n_jt;
-      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      const BlockPf cur = pf;
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_jt, p.bm);
+      const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
@@ -330,22 +385,23 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_jt, p.bm);
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int b = u / p.n_jt;
-      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      const BlockPf cur = pf;
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_jt, p.bm);
+      const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
-      const int64_t row0 = static_cast<int64_t>(b) * p.bm;
       const uint8_t* src[kGatherSlots];
       uint32_t dst[kGatherSlots];
       uint32_t live = 0;
 #pragma unroll
       for (int i = 0; i < kGatherSlots; ++i) {
-        const int r = 4 * g + 16 * i + (lane >> 3);
+        const int r = 4 * g + 16 * i + (lane >> 3);  // row id held by lane r % 32 in cur.id[r / 32 = i / 2]
+        const int id = __shfl_sync(0xffffffffu, cur.id[i >> 1], r & 31);
         dst[i] = static_cast<uint32_t>(r * kRowBytes + ((q ^ (r & 7)) << 4));
         src[i] = p.x;
         if (r < bi.nend && row_valid(bi, r)) {
-          const int t = __ldg(p.sorted_ids + row0 + r) / p.top_k;
-          src[i] = p.x + static_cast<int64_t>(t) * p.K * esize + q * 16;
+          src[i] = p.x + static_cast<int64_t>(id / p.top_k) * p.K * esize + q * 16;
           live |= 1u << i;
         }
       }
@@ -353,8 +409,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       const uint32_t sf_dst = static_cast<uint32_t>((lane & 31) * 16 + g * 4);  // row r = 32 g + lane
       if (kFp8) {
         const int r = 32 * g + lane;
-        if (r < bi.nend && row_valid(bi, r))
-          sf_src = p.x_sf + static_cast<int64_t>(__ldg(p.sorted_ids + row0 + r) / p.top_k) * KS;
+        if (r < bi.nend && row_valid(bi, r)) sf_src = p.x_sf + static_cast<int64_t>(pf_id(cur, g) / p.top_k) * KS;
       }
       for (int kc = 0; kc < n_kc; ++kc) {
         if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
@@ -378,9 +433,12 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     const int r = 32 * q + lane;
     int acc_it = 0;
     bool ok = true;
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_jt, p.bm);
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int b = u / p.n_jt, j = u - (u / p.n_jt) * p.n_jt;
-      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      const int b = u / n_jt, j = u - (u / n_jt) * n_jt;
+      const BlockPf cur = pf;
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_jt, p.bm);
+      const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
@@ -419,7 +477,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
               uint4* dst = reinterpret_cast<uint4*>(p.act + row * p.I + icol);
               dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
               dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-              p.act_sf[(static_cast<int64_t>(b) * p.n_jt + j) * kSfTileBytes + (r & 31) * 16 + (r >> 5) * 4 +
+              p.act_sf[(static_cast<int64_t>(b) * n_jt + j) * kSfTileBytes + (r & 31) * 16 + (r >> 5) * 4 +
                        (col0 >> 5)] = static_cast<uint8_t>(sc + 127);
             }
           } else if (mine && icol < p.I) {
@@ -499,7 +557,9 @@ __global__ void __launch_bounds__(kP2Threads, 1)
   const uint32_t tbase = *tmem_base_sm;
 
   const int n_blocks = num_blocks(p.ntpp, p.bm, p.max_blocks);
-  const int n_units = n_blocks * p.n_ht;
+  constexpr int TH = kTH;
+  const int n_ht = p.n_ht;
+  const int n_units = n_blocks * n_ht;
   constexpr int kKC = kFp8 ? 128 : 64;
   auto stage_ptr = [&](int s) { return smem + static_cast<size_t>(s) * p.stage_bytes; };
 
@@ -511,12 +571,15 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_ht, p.bm);
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int b = u / p.n_ht, ht = u - (u / p.n_ht) * p.n_ht;
-      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      const int b = u / n_ht, ht = u - (u / n_ht) * n_ht;
+      const BlockPf cur = pf;
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_ht, p.bm);
+      const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
-      const int nb = min(2, (p.K - ht * kTH) / 128);  // 128-row halves of this feature tile
-      const int w2_row = bi.e * p.K + ht * kTH;
+      const int nb = min(TH, p.K - ht * TH) / 128;  // 128-row pieces of this feature tile
+      const int w2_row = bi.e * p.K + ht * TH;
       const uint32_t tx = nb * 128 * kRowBytes + bi.n16 * kRowBytes + (kFp8 ? (1 + nb) * kSfTileBytes : 0);
       for (int kc = 0; kc < p.n_kc; ++kc) {
         if (lane == 0) {
@@ -533,7 +596,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
                         &full[s]);
               for (int i = 0; i < nb; ++i)
                 bulk_load(st + kOffSf + (1 + i) * kSfTileBytes,
-                          p.w2_sf + ((static_cast<int64_t>(bi.e) * MT2 + 2 * ht + i) * KT2 + kc) * kSfTileBytes,
+                          p.w2_sf + ((static_cast<int64_t>(bi.e) * MT2 + (ht * TH) / 128 + i) * KT2 + kc) * kSfTileBytes,
                           kSfTileBytes, &full[s]);
             }
           }
@@ -549,11 +612,14 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     uint32_t ph = 0;
     int acc_it = 0;
     bool ok = true;
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_ht, p.bm);
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int b = u / p.n_ht, ht = u - (u / p.n_ht) * p.n_ht;
-      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      const int ht = u - (u / n_ht) * n_ht;
+      const BlockPf cur = pf;
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_ht, p.bm);
+      const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
-      const int nn = min(kTH, p.K - ht * kTH);
+      const int nn = min(TH, p.K - ht * TH);
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
       if (lane == 0) ok = mbar_wait(&acc_empty[buf], acc_ph ^ 1u, abort_flag, p.status);
@@ -606,18 +672,20 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     uint4* stg4 = reinterpret_cast<uint4*>(ctrl + kP2Ctrl) + (warp - kP2FirstEpi) * (kStageFloatsPerWarp / 4);
     int acc_it = 0;
     bool ok = true;
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_ht, p.bm);
     for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int b = u / p.n_ht, ht = u - (u / p.n_ht) * p.n_ht;
-      const BlockInfo bi = block_info(p.sorted_ids, p.expert_ids, b, p.bm, p.R, p.E);
+      const int ht = u - (u / n_ht) * n_ht;
+      const BlockPf cur = pf;
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_ht, p.bm);
+      const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
-      const int nn = min(kTH, p.K - ht * kTH);
-      const int64_t row0 = static_cast<int64_t>(b) * p.bm;
+      const int nn = min(TH, p.K - ht * TH);
       // the route and its weight, fetched while the MMAs run
       const bool mine = row_valid(bi, r);
       int route = 0;
       float wgt = 0.f;
       if (mine) {
-        route = __ldg(p.sorted_ids + row0 + r);
+        route = pf_id(cur, q);
         wgt = __ldg(p.topk_w + route);
       }
       const int buf = acc_it % kNumAcc;
@@ -637,7 +705,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
         // weighted rows in fp32 (16 columns per slice); the mxfp8 path rounds
         // them to bf16 (32 columns per slice), half the bytes.
         const int half = nn / 2;
-        const int64_t col_base = static_cast<int64_t>(ht) * kTH + h * half;
+        const int64_t col_base = static_cast<int64_t>(ht) * TH + h * half;
 #pragma unroll 1
         for (int c = 0; c < half; c += 32) {
           uint32_t yr[32];
