@@ -88,6 +88,7 @@ struct P1Params {
   int* status;
   int K, N, I, E, top_k, bm, R;
   int max_blocks;           // blocks a kernel may visit
+  int w_reuse;              // 1: experts average more than one planner block (weights re-read)
   int n_jt;                 // ceil(I / 128): work units per planner block
   int stages, stage_bytes;
 };
@@ -104,6 +105,7 @@ struct P2Params {
   int* status;
   int K, I, E, top_k, bm, R;
   int max_blocks;
+  int w_reuse;
   int n_ht;                 // ceil(K / 256): work units per planner block
   int n_kc;                 // K-chunks of the down GEMM
   int stages, stage_bytes;
@@ -273,7 +275,11 @@ __global__ void __launch_bounds__(kP1Threads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer (weights)
-    const uint64_t pol = policy_evict_first();
+    // A weight tile is read by every planner block of its expert: when
+    // experts average more than one block (large T) those reads come close
+    // together, so the tiles keep normal L2 priority; otherwise each is read
+    // once and is evicted first.
+    const uint64_t pol = p.w_reuse ? policy_evict_normal() : policy_evict_first();
     const uint32_t tx = 2 * kTI * kRowBytes + (kFp8 ? 2 * kSfTileBytes : 0);
     const int MT1 = p.N / 128, KT1 = p.K / 128;
     int s = 0;
@@ -565,7 +571,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
-    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_w = p.w_reuse ? policy_evict_normal() : policy_evict_first();  // as in the gate/up phase
     const uint64_t pol_a = policy_evict_last();
     const int MT2 = p.K / 128, KT2 = p.I / 128;
     int s = 0;
@@ -992,6 +998,7 @@ static int run_fused(const FusedArgs& a) {
   p1.K = a.K; p1.N = a.N; p1.I = I; p1.E = a.E; p1.top_k = a.top_k; p1.bm = a.bm;
   p1.R = a.T * a.top_k;
   p1.max_blocks = max_blocks;
+  p1.w_reuse = static_cast<int64_t>(a.T) * a.top_k >= static_cast<int64_t>(a.E) * a.bm ? 1 : 0;
   p1.n_jt = (I + kTI - 1) / kTI;
   p1.stage_bytes = stage_bytes(a.fp8);
   p1.stages = pick_stages(p1.stage_bytes, kP1Ctrl, req_stages, 8);
@@ -1008,6 +1015,7 @@ static int run_fused(const FusedArgs& a) {
   p2.status = p1.status;
   p2.K = a.K; p2.I = I; p2.E = a.E; p2.top_k = a.top_k; p2.bm = a.bm; p2.R = p1.R;
   p2.max_blocks = max_blocks;
+  p2.w_reuse = p1.w_reuse;
   p2.n_ht = (a.K + kTH - 1) / kTH;
   p2.n_kc = a.fp8 ? I / 128 : (I + 63) / 64;
   p2.stage_bytes = stage_bytes(a.fp8);
