@@ -296,17 +296,22 @@ class Problem:
 
 def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barrier=None, sample_clocks=True,
             local: int = 0):
-    """Device time of `steps` steps after `warmup`.  With flush_l2 every step is
+    """Device time of `steps` steps after `warmup`.
+
+    Pass 1 (the reported time): the steps run with nothing between their
+    launches, so the library's programmatic dependent launch overlaps each
+    kernel's prologue with the previous kernel.  With flush_l2 every step is
     bracketed by its own events and a >L2 buffer is written between steps
     (outside the timed windows); otherwise the steps run back to back between
-    one pair of events.  The library's phase events time each kernel."""
+    one pair of events.
+    Pass 2 (the per-kernel breakdown): the same steps with the library's phase
+    events recorded between its launches (events between launches can keep the
+    launches from overlapping, so pass 2 is used for the per-kernel times only).
+    """
     import torch
 
     moe = prob.moe
     stream = torch.cuda.current_stream()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
-    pev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    tunes = [moe.Tuning.with_events(e, prob.stages, prob.ctas) for e in ev]
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=prob.dev) if flush_l2 else None
     for _ in range(max(3, warmup)):
         prob.step()
@@ -320,27 +325,34 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
     if clocks:
         clocks.start()
         time.sleep(0.3)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)] \
-        if flush_l2 else None
-    t0.record(stream)
-    for i in range(steps):
-        if s_ev:
-            s_ev[i][0].record(stream)
-        prob.step(tunes[i], pev[i])
-        if s_ev:
-            s_ev[i][1].record(stream)
-            flush.fill_(1)
-    t1.record(stream)
-    torch.cuda.synchronize()
+
+    def timed(tunes=None, pev=None):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)] \
+            if flush_l2 else None
+        t0.record(stream)
+        for i in range(steps):
+            if s_ev:
+                s_ev[i][0].record(stream)
+            prob.step(None if tunes is None else tunes[i], None if pev is None else pev[i])
+            if s_ev:
+                s_ev[i][1].record(stream)
+                flush.fill_(1)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in s_ev) if s_ev else t0.elapsed_time(t1)
+
+    total_ms = timed()
     if barrier:
         barrier()
     clk = clocks.stop() if clocks else None
     moe.moe_device_status()
-    if s_ev:
-        total_ms = sum(a.elapsed_time(b) for a, b in s_ev)
-    else:
-        total_ms = t0.elapsed_time(t1)
+    # pass 2: per-kernel times
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    pev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    tunes = [moe.Tuning.with_events(e, prob.stages, prob.ctas) for e in ev]
+    timed(tunes, pev)
+    moe.moe_device_status()
     return {"total_ms": total_ms, "ms_step": total_ms / steps,
             "plan_ms": sum(a.elapsed_time(e[0]) for a, e in zip(pev, ev)) / steps,
             "p1_ms": sum(e[0].elapsed_time(e[1]) for e in ev) / steps,

@@ -237,9 +237,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
   constexpr int kNumAcc = kFp8 ? 1 : 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // clear the route flags (phase 2 sets them); nothing reads them in this phase
-  for (int i = blockIdx.x * kP1Threads + threadIdx.x; i < p.R; i += gridDim.x * kP1Threads) p.flags[i] = 0;
-
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       // producer lane 0 (with the TMA byte count) + the cp.async completion
@@ -263,6 +261,10 @@ __global__ void __launch_bounds__(kP1Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_base_sm;
+  // everything above overlaps the planner; its outputs are read below
+  pdl_wait();
+  // clear the route flags (phase 2 sets them); nothing reads them in this phase
+  for (int i = blockIdx.x * kP1Threads + threadIdx.x; i < p.R; i += gridDim.x * kP1Threads) p.flags[i] = 0;
 
   const int n_blocks = num_blocks(p.ntpp, p.bm, p.max_blocks);
   const int n_jt = p.n_jt;
@@ -539,6 +541,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 
   constexpr int kNumAcc = kFp8 ? 1 : 2;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
@@ -561,6 +564,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_base_sm;
+  pdl_wait();  // the gate/up phase's intermediate is read below
 
   const int n_blocks = num_blocks(p.ntpp, p.bm, p.max_blocks);
   constexpr int TH = kTH;
@@ -790,9 +794,15 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
   }
 }
 
-template <typename TP>
-__global__ void moe_combine_kernel(const TP* __restrict__ yw, const int32_t* __restrict__ flags,
-                                   __nv_bfloat16* __restrict__ out, int T, int K, int top_k) {
+// One thread sums 8 consecutive features of one token over its top_k routes.
+// The route flags and every route's 8 partials are loaded before any of them
+// is used (the loads of a route whose flag is 0 read workspace bytes that are
+// then discarded), so a thread has all its loads in flight at once; the sum
+// runs in route order, so the result does not depend on scheduling.
+template <typename TP, int kMaxK>
+__global__ void __launch_bounds__(256) moe_combine_kernel(const TP* __restrict__ yw, const int32_t* __restrict__ flags,
+                                                          __nv_bfloat16* __restrict__ out, int T, int K, int top_k) {
+  pdl_wait();  // the down phase's partial rows are read below
   const int kv = K / 8;
   const int64_t n = static_cast<int64_t>(T) * kv;
   for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n;
@@ -800,14 +810,24 @@ __global__ void moe_combine_kernel(const TP* __restrict__ yw, const int32_t* __r
     const int64_t t = v / kv;
     const int h = static_cast<int>(v - t * kv) * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < top_k; ++j) {
-      const int64_t r = t * top_k + j;
-      if (__ldg(flags + r)) {
-        float y[8];
-        load8(yw + r * K + h, y);
+    for (int j0 = 0; j0 < top_k; j0 += kMaxK) {
+      int f[kMaxK];
+      float y[kMaxK][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] += y[i];
+      for (int j = 0; j < kMaxK; ++j) {
+        f[j] = 0;
+        if (j0 + j < top_k) {
+          const int64_t r = t * top_k + j0 + j;
+          f[j] = __ldg(flags + r);
+          load8(yw + r * K + h, y[j]);
+        }
       }
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j)
+        if (f[j]) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] += y[j][i];
+        }
     }
     __nv_bfloat162 o[4];
 #pragma unroll
@@ -1046,28 +1066,44 @@ static int run_fused(const FusedArgs& a) {
     if ((rc = set_smem_attr(moe_p1_kernel<false>, smem1, attr_done[2])) != MOE_OK) return rc;
     if ((rc = set_smem_attr(moe_p2_kernel<false>, smem2, attr_done[3])) != MOE_OK) return rc;
   }
+  // The three launches are chained by programmatic dependent launch: each
+  // kernel lets the next one be scheduled early (prologue: barriers, TMEM,
+  // tensor-map prefetch) and the next one waits (griddepcontrol.wait) before
+  // reading the previous one's results.
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  auto config = [&](int grid, int threads, int smem) {
+    cudaLaunchConfig_t c = {};
+    c.gridDim = dim3(grid, 1, 1);
+    c.blockDim = dim3(threads, 1, 1);
+    c.dynamicSmemBytes = smem;
+    c.stream = a.stream;
+    c.attrs = pdl;
+    c.numAttrs = 1;
+    return c;
+  };
   if ((rc = mark(0)) != MOE_OK) return rc;
-  if (a.fp8) moe_p1_kernel<true><<<grid1, kP1Threads, smem1, a.stream>>>(tm_w1, p1);
-  else moe_p1_kernel<false><<<grid1, kP1Threads, smem1, a.stream>>>(tm_w1, p1);
-  cudaError_t err = cudaGetLastError();
+  cudaLaunchConfig_t c1 = config(grid1, kP1Threads, smem1);
+  cudaError_t err = a.fp8 ? cudaLaunchKernelEx(&c1, moe_p1_kernel<true>, tm_w1, p1)
+                          : cudaLaunchKernelEx(&c1, moe_p1_kernel<false>, tm_w1, p1);
   if (err != cudaSuccess) return cuda_fail("fused_moe: gate/up phase launch", err);
   if ((rc = mark(1)) != MOE_OK) return rc;
-  if (a.fp8) moe_p2_kernel<true><<<grid2, kP2Threads, smem2, a.stream>>>(tm_w2, tm_act, p2);
-  else moe_p2_kernel<false><<<grid2, kP2Threads, smem2, a.stream>>>(tm_w2, tm_act, p2);
-  err = cudaGetLastError();
+  cudaLaunchConfig_t c2 = config(grid2, kP2Threads, smem2);
+  err = a.fp8 ? cudaLaunchKernelEx(&c2, moe_p2_kernel<true>, tm_w2, tm_act, p2)
+              : cudaLaunchKernelEx(&c2, moe_p2_kernel<false>, tm_w2, tm_act, p2);
   if (err != cudaSuccess) return cuda_fail("fused_moe: down phase launch", err);
   if ((rc = mark(2)) != MOE_OK) return rc;
   const int64_t nvec = static_cast<int64_t>(a.T) * (a.K / 8);
   const int64_t cblocks = (nvec + 255) / 256;
-  const int cgrid = static_cast<int>(cblocks < 4L * nsm ? cblocks : 4L * nsm);
-  if (a.fp8)
-    moe_combine_kernel<__nv_bfloat16><<<cgrid, 256, 0, a.stream>>>(
-        reinterpret_cast<const __nv_bfloat16*>(ws + L.yw), p1.flags, static_cast<__nv_bfloat16*>(a.out), a.T, a.K,
-        a.top_k);
-  else
-    moe_combine_kernel<float><<<cgrid, 256, 0, a.stream>>>(reinterpret_cast<const float*>(ws + L.yw), p1.flags,
-                                                           static_cast<__nv_bfloat16*>(a.out), a.T, a.K, a.top_k);
-  err = cudaGetLastError();
+  const int cgrid = static_cast<int>(cblocks < 8L * nsm ? cblocks : 8L * nsm);
+  cudaLaunchConfig_t c3 = config(cgrid, 256, 0);
+  __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(a.out);
+  err = a.fp8 ? cudaLaunchKernelEx(&c3, moe_combine_kernel<__nv_bfloat16, 8>,
+                                   reinterpret_cast<const __nv_bfloat16*>(ws + L.yw),
+                                   static_cast<const int32_t*>(p1.flags), outp, a.T, a.K, a.top_k)
+              : cudaLaunchKernelEx(&c3, moe_combine_kernel<float, 8>, reinterpret_cast<const float*>(ws + L.yw),
+                                   static_cast<const int32_t*>(p1.flags), outp, a.T, a.K, a.top_k);
   if (err != cudaSuccess) return cuda_fail("fused_moe: combine launch", err);
   return mark(3);
 }

@@ -33,6 +33,7 @@
 // and expert_ids is filled block by block; these writes are spread over the
 // cluster's CTAs.
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace moe {
 
@@ -84,6 +85,7 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
   int32_t* warp_tot = off + E + 1;            // [kAlignWarps]
   uint16_t* ids16 = reinterpret_cast<uint16_t*>(warp_tot + kAlignWarps);  // [chunk] when staged
 
+  pdl_launch_dependents();  // the fused phases may start their prologue now
   const uint32_t crank = cluster_ctarank(), csize = cluster_nctarank();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cchunk = (R + static_cast<int>(csize) - 1) / static_cast<int>(csize);

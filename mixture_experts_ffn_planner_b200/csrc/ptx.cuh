@@ -276,6 +276,16 @@ __host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sfa_id,
          (static_cast<uint32_t>(M >> 4) << 24) | (sfa_id << 29);
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// Lets the next kernel on the stream (launched with programmatic stream
+// serialisation) be scheduled before this one finishes.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Blocks until the preceding kernel(s) on the stream have completed and their
+// memory is visible; a no-op when the kernel was launched normally.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------- misc
 // silu(g) = g / (1 + e^-g) with the fast exponential and fast division
 // intrinsics (relative error a few ulp of fp32, far below the bf16 / e4m3
