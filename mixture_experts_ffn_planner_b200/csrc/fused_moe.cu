@@ -71,9 +71,12 @@ constexpr int kP2Ctrl = 64 * 16 + 16;
 constexpr int kStageFloatsPerWarp = 32 * 16;
 constexpr int kP2Staging = kEpiWarps * kStageFloatsPerWarp * 4;
 
-// Stage layout (both phases): [A 128 rows x 128 B][B 256 rows x 128 B][SFA 512][SFB 2 x 512]
-constexpr int kOffB = kM * kRowBytes;
-constexpr int kOffSf = kOffB + 2 * 128 * kRowBytes;
+// Stage layout (both phases): [A a_rows x 128 B][B 256 rows x 128 B][SFA 512][SFB 2 x 512].
+// a_rows (a multiple of 16, at most 128) bounds the routed rows of any
+// planner block -- min(block_m, T * top_k) -- so small batches get a small A
+// region and more pipeline stages (more weight bytes in flight per SM).  The
+// MMA still reads 128 A rows; the rows past a_rows belong to the B region and
+// only produce accumulator rows that are never read.
 
 struct P1Params {
   const uint8_t* x;         // (T, K) bf16 or e4m3
@@ -91,6 +94,7 @@ struct P1Params {
   int w_reuse;              // 1: experts average more than one planner block (weights re-read)
   int n_jt;                 // ceil(I / 128): work units per planner block
   int stages, stage_bytes;
+  int off_b, off_sf;        // stage offsets of the B tile and of the scale tiles
 };
 
 struct P2Params {
@@ -109,6 +113,7 @@ struct P2Params {
   int n_ht;                 // ceil(K / 256): work units per planner block
   int n_kc;                 // K-chunks of the down GEMM
   int stages, stage_bytes;
+  int off_b, off_sf;
 };
 
 // Per-unit facts every warp role derives the same way (warp-collective).
@@ -302,14 +307,14 @@ __global__ void __launch_bounds__(kP1Threads, 1)
           if (ok) {
             uint8_t* st = stage_ptr(s);
             mbar_arrive_expect_tx(&full[s], tx);
-            tma_load_2d(st + kOffB, &tm_w1, &full[s], kc * kKC, gate_row, pol);
-            tma_load_2d(st + kOffB + 128 * kRowBytes, &tm_w1, &full[s], kc * kKC, up_row, pol);
+            tma_load_2d(st + p.off_b, &tm_w1, &full[s], kc * kKC, gate_row, pol);
+            tma_load_2d(st + p.off_b + 128 * kRowBytes, &tm_w1, &full[s], kc * kKC, up_row, pol);
             if (kFp8) {
               const uint8_t* sfg = p.w1_sf + ((static_cast<int64_t>(bi.e) * MT1 + j) * KT1 + kc) * kSfTileBytes;
               const uint8_t* sfu =
                   p.w1_sf + ((static_cast<int64_t>(bi.e) * MT1 + p.I / 128 + j) * KT1 + kc) * kSfTileBytes;
-              bulk_load(st + kOffSf + kSfTileBytes, sfg, kSfTileBytes, &full[s]);
-              bulk_load(st + kOffSf + 2 * kSfTileBytes, sfu, kSfTileBytes, &full[s]);
+              bulk_load(st + p.off_sf + kSfTileBytes, sfg, kSfTileBytes, &full[s]);
+              bulk_load(st + p.off_sf + 2 * kSfTileBytes, sfu, kSfTileBytes, &full[s]);
             }
           }
         }
@@ -348,11 +353,11 @@ __global__ void __launch_bounds__(kP1Threads, 1)
             fence_proxy_async_smem();
             uint8_t* st = stage_ptr(s);
             const uint64_t ad = sdesc_sw128(smem_u32(st));
-            const uint64_t bd = sdesc_sw128(smem_u32(st + kOffB));
+            const uint64_t bd = sdesc_sw128(smem_u32(st + p.off_b));
             if (kFp8) {
-              tc_cp_32x128b_x4(tbase + kSfaCol, sdesc_sf(smem_u32(st + kOffSf)));
-              tc_cp_32x128b_x4(tbase + kSfbCol, sdesc_sf(smem_u32(st + kOffSf + kSfTileBytes)));
-              tc_cp_32x128b_x4(tbase + kSfbCol + 4, sdesc_sf(smem_u32(st + kOffSf + 2 * kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + kSfaCol, sdesc_sf(smem_u32(st + p.off_sf)));
+              tc_cp_32x128b_x4(tbase + kSfbCol, sdesc_sf(smem_u32(st + p.off_sf + kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + kSfbCol + 4, sdesc_sf(smem_u32(st + p.off_sf + 2 * kSfTileBytes)));
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -427,7 +432,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
 #pragma unroll
         for (int i = 0; i < kGatherSlots; ++i)
           if (live & (1u << i)) cp_async_16(abase + dst[i], src[i] + kc * kRowBytes);
-        if (kFp8 && sf_src) cp_async_4(abase + kOffSf + sf_dst, sf_src + 4 * kc);
+        if (kFp8 && sf_src) cp_async_4(abase + p.off_sf + sf_dst, sf_src + 4 * kc);
         cp_async_mbar_arrive(&full[s]);
         if (++s == S) { s = 0; ph ^= 1u; }
       }
@@ -600,12 +605,12 @@ __global__ void __launch_bounds__(kP2Threads, 1)
             for (int i = 0; i < bi.n16 / 16; ++i)
               tma_load_2d(st + i * 16 * kRowBytes, &tm_act, &full[s], kc * kKC, b * p.bm + 16 * i, pol_a);
             for (int i = 0; i < nb; ++i)
-              tma_load_2d(st + kOffB + i * 128 * kRowBytes, &tm_w2, &full[s], kc * kKC, w2_row + 128 * i, pol_w);
+              tma_load_2d(st + p.off_b + i * 128 * kRowBytes, &tm_w2, &full[s], kc * kKC, w2_row + 128 * i, pol_w);
             if (kFp8) {
-              bulk_load(st + kOffSf, p.act_sf + (static_cast<int64_t>(b) * KT2 + kc) * kSfTileBytes, kSfTileBytes,
+              bulk_load(st + p.off_sf, p.act_sf + (static_cast<int64_t>(b) * KT2 + kc) * kSfTileBytes, kSfTileBytes,
                         &full[s]);
               for (int i = 0; i < nb; ++i)
-                bulk_load(st + kOffSf + (1 + i) * kSfTileBytes,
+                bulk_load(st + p.off_sf + (1 + i) * kSfTileBytes,
                           p.w2_sf + ((static_cast<int64_t>(bi.e) * MT2 + (ht * TH) / 128 + i) * KT2 + kc) * kSfTileBytes,
                           kSfTileBytes, &full[s]);
             }
@@ -644,11 +649,11 @@ __global__ void __launch_bounds__(kP2Threads, 1)
             tc_fence_after();
             uint8_t* st = stage_ptr(s);
             const uint64_t ad = sdesc_sw128(smem_u32(st));
-            const uint64_t bd = sdesc_sw128(smem_u32(st + kOffB));
+            const uint64_t bd = sdesc_sw128(smem_u32(st + p.off_b));
             if (kFp8) {
-              tc_cp_32x128b_x4(tbase + kSfaCol, sdesc_sf(smem_u32(st + kOffSf)));
-              tc_cp_32x128b_x4(tbase + kSfbCol, sdesc_sf(smem_u32(st + kOffSf + kSfTileBytes)));
-              tc_cp_32x128b_x4(tbase + kSfbCol + 4, sdesc_sf(smem_u32(st + kOffSf + 2 * kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + kSfaCol, sdesc_sf(smem_u32(st + p.off_sf)));
+              tc_cp_32x128b_x4(tbase + kSfbCol, sdesc_sf(smem_u32(st + p.off_sf + kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + kSfbCol + 4, sdesc_sf(smem_u32(st + p.off_sf + 2 * kSfTileBytes)));
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -934,8 +939,14 @@ struct FusedArgs {
   cudaStream_t stream;
 };
 
-static int stage_bytes(bool fp8) {
-  return static_cast<int>(round_up(kOffSf + (fp8 ? 3 * kSfTileBytes : 0), 1024));
+static int a_region_rows(int bm, int64_t R) {
+  const int64_t r = std::min<int64_t>(bm, R);
+  return static_cast<int>(std::min<int64_t>(kM, round_up(std::max<int64_t>(r, 1), 16)));
+}
+static int off_b_of(int a_rows) { return static_cast<int>(round_up(static_cast<int64_t>(a_rows) * kRowBytes, 1024)); }
+static int off_sf_of(int a_rows) { return off_b_of(a_rows) + 2 * 128 * kRowBytes; }
+static int stage_bytes(bool fp8, int a_rows) {
+  return static_cast<int>(round_up(off_sf_of(a_rows) + (fp8 ? 3 * kSfTileBytes : 0), 1024));
 }
 constexpr int kP1Ctrl = 64 * 16 + 16;  // barriers, tmem base, abort flag
 
@@ -1020,7 +1031,10 @@ static int run_fused(const FusedArgs& a) {
   p1.max_blocks = max_blocks;
   p1.w_reuse = static_cast<int64_t>(a.T) * a.top_k >= static_cast<int64_t>(a.E) * a.bm ? 1 : 0;
   p1.n_jt = (I + kTI - 1) / kTI;
-  p1.stage_bytes = stage_bytes(a.fp8);
+  const int a_rows = a_region_rows(a.bm, static_cast<int64_t>(a.T) * a.top_k);
+  p1.stage_bytes = stage_bytes(a.fp8, a_rows);
+  p1.off_b = off_b_of(a_rows);
+  p1.off_sf = off_sf_of(a_rows);
   p1.stages = pick_stages(p1.stage_bytes, kP1Ctrl, req_stages, 8);
 
   P2Params p2{};
@@ -1038,7 +1052,9 @@ static int run_fused(const FusedArgs& a) {
   p2.w_reuse = p1.w_reuse;
   p2.n_ht = (a.K + kTH - 1) / kTH;
   p2.n_kc = a.fp8 ? I / 128 : (I + 63) / 64;
-  p2.stage_bytes = stage_bytes(a.fp8);
+  p2.stage_bytes = stage_bytes(a.fp8, a_rows);
+  p2.off_b = p1.off_b;
+  p2.off_sf = p1.off_sf;
   p2.stages = pick_stages(p2.stage_bytes, kP2Ctrl + kP2Staging, req_stages, 8);
   if (p1.stages < 2 || p2.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "%s: shared memory too small", nm);
 
