@@ -312,11 +312,19 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
 
     moe = prob.moe
     stream = torch.cuda.current_stream()
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=prob.dev) if flush_l2 else None
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=prob.dev) if flush_l2 else None
+
+    def flush():
+        # write a buffer 4x the L2 size, then read it back: the read evicts the
+        # dirty lines the write left (their write-back happens here, outside
+        # the timed window) so the next step starts with a cold, clean L2
+        flush_buf.fill_(1)
+        flush_buf.max()
+
     for _ in range(max(3, warmup)):
         prob.step()
-        if flush is not None:
-            flush.fill_(1)
+        if flush_buf is not None:
+            flush()
     moe.moe_device_status()
     if barrier:
         barrier()
@@ -337,7 +345,7 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
             prob.step(None if tunes is None else tunes[i], None if pev is None else pev[i])
             if s_ev:
                 s_ev[i][1].record(stream)
-                flush.fill_(1)
+                flush()
         t1.record(stream)
         torch.cuda.synchronize()
         return sum(a.elapsed_time(b) for a, b in s_ev) if s_ev else t0.elapsed_time(t1)
@@ -420,7 +428,7 @@ def roofline_of_p1(sh: W.Shape, cm: dict, p1_ms: float, peaks: dict, peak_src: s
 
 def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
     ms_step = m["ms_step"]
-    l2 = ("L2 flushed between steps (512 MB write outside the per-step events)" if flush_l2 else
+    l2 = ("L2 flushed between steps (512 MB written then read back, outside the per-step events)" if flush_l2 else
           f"inputs larger than L2 (touched expert weights {cm['bytes_w'] / 1e9:.2f} GB per step)")
     return {
         "metric": METRIC, "value": world * cm["flops"] / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",

@@ -47,6 +47,14 @@ __device__ int g_moe_status = 0;
 
 constexpr int kM = 128;           // MMA M: routed rows of one planner block (rows >= block_m unused)
 constexpr int kTI = 128;          // intermediate columns per gate/up unit (gate 128 + up 128 = MMA N 256)
+// Split-K of the gate/up phase for small problems: when there are fewer work
+// units than half the CTAs, a unit whose block has at most kSplitRows routed
+// rows is cut into up to kMaxSplit K-ranges, each on its own CTA; the fp32
+// partial accumulators go to the workspace and moe_p1_reduce_kernel sums them
+// (in split order) and applies SwiGLU.
+constexpr int kSplitRows = 32;
+constexpr int kMaxSplit = 8;
+constexpr int kMaxSplitItems = 256;  // bounds the partial workspace
 constexpr int kTH = 256;          // output features per down unit (MMA N)
 constexpr int kRowBytes = 128;    // bytes of one operand row per pipeline stage
 constexpr int kSfTileBytes = 512; // one blocked scale tile: 128 rows x 4 scales
@@ -92,6 +100,7 @@ struct P1Params {
   int K, N, I, E, top_k, bm, R;
   int max_blocks;           // blocks a kernel may visit
   int w_reuse;              // 1: experts average more than one planner block (weights re-read)
+  float* part;              // split-K partials: [kMaxSplitItems][kSplitRows][256] fp32
   int n_jt;                 // ceil(I / 128): work units per planner block
   int stages, stage_bytes;
   int off_b, off_sf;        // stage offsets of the B tile and of the scale tiles
@@ -195,6 +204,15 @@ __device__ __forceinline__ int pf_id(const BlockPf& f, int q) {
   return q == 0 ? f.id[0] : q == 1 ? f.id[1] : q == 2 ? f.id[2] : f.id[3];
 }
 
+// Number of K-splits per gate/up unit (1: no split), identical in every CTA
+// and in the reduction kernel.
+__device__ __forceinline__ int split_count(int n_units, int grid, int n_kc) {
+  if (n_units <= 0 || 2 * n_units > grid) return 1;
+  int sk = min(min(grid, kMaxSplitItems) / n_units, kMaxSplit);
+  sk = min(sk, n_kc / 2);
+  return max(sk, 1);
+}
+
 __device__ __forceinline__ bool row_valid(const BlockInfo& bi, int c) {
   return (bi.vm[c >> 5] >> (c & 31)) & 1u;
 }
@@ -277,6 +295,22 @@ __global__ void __launch_bounds__(kP1Threads, 1)
   constexpr int kKC = kFp8 ? 128 : 64;  // K elements per stage (128 bytes per row)
   const int n_kc = p.K / kKC;
   const int esize = kFp8 ? 1 : 2;
+  // Work items: (unit, K-split).  Without splitting an item is a unit.
+  const int nsplit = split_count(n_units, gridDim.x, n_kc);
+  const int n_items = n_units * nsplit;
+  const int per_block = n_jt * nsplit;  // items per planner block
+  // k-range of item w (whose block has bi.nend rows); empty when the item is
+  // a non-first split of a unit that is not split.
+  auto krange = [&](int w, const BlockInfo& bi, int& k0, int& k1) {
+    const int sidx = w % nsplit;
+    if (nsplit > 1 && bi.nend <= kSplitRows) {
+      k0 = sidx * n_kc / nsplit;
+      k1 = (sidx + 1) * n_kc / nsplit;
+    } else {
+      k0 = 0;
+      k1 = sidx == 0 ? n_kc : 0;
+    }
+  };
 
   auto stage_ptr = [&](int s) { return smem + static_cast<size_t>(s) * p.stage_bytes; };
 
@@ -292,16 +326,20 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_jt, p.bm);
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_items, per_block, p.bm);
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      const int u = w / nsplit;
       const int j = u - (u / n_jt) * n_jt;
       const BlockPf cur = pf;
-      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_jt, p.bm);
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, w + gridDim.x, n_items, per_block, p.bm);
       const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
+      int k0, k1;
+      krange(w, bi, k0, k1);
+      if (k0 == k1) continue;
       const int gate_row = bi.e * p.N + j * kTI;
       const int up_row = bi.e * p.N + p.I + j * kTI;
-      for (int kc = 0; kc < n_kc; ++kc) {
+      for (int kc = k0; kc < k1; ++kc) {
         if (lane == 0) {
           ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
           if (ok) {
@@ -330,12 +368,15 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     uint32_t ph = 0;
     int acc_it = 0;
     bool ok = true;
-    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_jt, p.bm);
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_items, per_block, p.bm);
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
       const BlockPf cur = pf;
-      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_jt, p.bm);
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, w + gridDim.x, n_items, per_block, p.bm);
       const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
+      int k0, k1;
+      krange(w, bi, k0, k1);
+      if (k0 == k1) continue;
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
       if (lane == 0) ok = mbar_wait(&acc_empty[buf], acc_ph ^ 1u, abort_flag, p.status);
@@ -343,7 +384,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t d = tbase + static_cast<uint32_t>(buf) * 256u;
-      for (int kc = 0; kc < n_kc; ++kc) {
+      for (int kc = k0; kc < k1; ++kc) {
         if (lane == 0) {
           ok = mbar_wait(&full[s], ph, abort_flag, p.status);
           if (ok) {
@@ -361,7 +402,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (kc | kk) != 0;
+              const uint32_t acc = (kc != k0 || kk != 0) ? 1u : 0u;
               const uint64_t step = static_cast<uint64_t>(2 * kk);  // 32 bytes along K
               if (kFp8) {
                 const uint32_t sfid = static_cast<uint32_t>(kk) << 30;
@@ -398,12 +439,15 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_jt, p.bm);
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_items, per_block, p.bm);
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
       const BlockPf cur = pf;
-      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_jt, p.bm);
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, w + gridDim.x, n_items, per_block, p.bm);
       const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
+      int k0, k1;
+      krange(w, bi, k0, k1);
+      if (k0 == k1) continue;
       const uint8_t* src[kGatherSlots];
       uint32_t dst[kGatherSlots];
       uint32_t live = 0;
@@ -424,7 +468,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
         const int r = 32 * g + lane;
         if (r < bi.nend && row_valid(bi, r)) sf_src = p.x_sf + static_cast<int64_t>(pf_id(cur, g) / p.top_k) * KS;
       }
-      for (int kc = 0; kc < n_kc; ++kc) {
+      for (int kc = k0; kc < k1; ++kc) {
         if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
@@ -446,13 +490,17 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     const int r = 32 * q + lane;
     int acc_it = 0;
     bool ok = true;
-    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_jt, p.bm);
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_items, per_block, p.bm);
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      const int u = w / nsplit;
       const int b = u / n_jt, j = u - (u / n_jt) * n_jt;
       const BlockPf cur = pf;
-      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_jt, p.bm);
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, w + gridDim.x, n_items, per_block, p.bm);
       const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
+      int k0, k1;
+      krange(w, bi, k0, k1);
+      if (k0 == k1) continue;
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
       ok = mbar_wait(&acc_full[buf], acc_ph, abort_flag, p.status);
@@ -462,7 +510,27 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       const bool mine = row_valid(bi, r);
       const int64_t row = static_cast<int64_t>(b) * p.bm + r;
       const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 256u;
-      if (32 * q < bi.nend) {  // warp-uniform: skip quadrants with no routed row
+      if (nsplit > 1 && bi.nend <= kSplitRows) {
+        // split item: hand the raw gate/up partials (rows < 32, quadrant 0)
+        // to the reduction kernel
+        if (q == 0) {
+          float* dst_row = p.part + (static_cast<int64_t>(w) * kSplitRows + r) * 256;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            const int col = (c < 2 ? 0 : 128) + 64 * h + 32 * (c & 1);  // gate halves, then up halves
+            uint32_t v[32];
+            tmem_ld32(tacc + col, v);
+            tmem_ld_wait();
+            if (mine) {
+              float4* d4 = reinterpret_cast<float4*>(dst_row + col);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                    __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            }
+          }
+        }
+      } else if (32 * q < bi.nend) {  // warp-uniform: skip quadrants with no routed row
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           const int col0 = 64 * h + 32 * c;  // within the unit's 128-column tile
@@ -523,6 +591,70 @@ __global__ void __launch_bounds__(kP1Threads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
+  }
+}
+
+// ========================================================================
+// split-K reduction of the gate/up phase (small problems only)
+// ========================================================================
+// One warp per (split unit, row): lane l sums columns 4l..4l+3 of the
+// gate and up partials over the splits in split order (deterministic),
+// applies SwiGLU and writes the intermediate exactly as the gate/up epilogue
+// does (bf16, or e4m3 codes with one e8m0 scale per 32 columns -- the amax of
+// a 32-column block is reduced over its 8 lanes).
+template <bool kFp8>
+__global__ void __launch_bounds__(256) moe_p1_reduce_kernel(const __grid_constant__ P1Params p, int grid1) {
+  pdl_launch_dependents();
+  pdl_wait();  // the gate/up phase's partials are read below
+  const int n_blocks = num_blocks(p.ntpp, p.bm, p.max_blocks);
+  const int n_units = n_blocks * p.n_jt;
+  constexpr int kKC = kFp8 ? 128 : 64;
+  const int nsplit = split_count(n_units, grid1, p.K / kKC);
+  if (nsplit <= 1) return;
+  const int lane = threadIdx.x & 31;
+  const int gw = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int nw = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+  for (int task = gw; task < n_units * kSplitRows; task += nw) {
+    const int u = task / kSplitRows, r = task - (task / kSplitRows) * kSplitRows;
+    const int b = u / p.n_jt, j = u - (u / p.n_jt) * p.n_jt;
+    const BlockInfo bi = block_finalize(block_prefetch(p.sorted_ids, p.expert_ids, b, n_blocks, 1, p.bm), p.R, p.E);
+    if (bi.nend == 0 || bi.nend > kSplitRows || r >= bi.nend || !row_valid(bi, r)) continue;  // warp-uniform
+    float g[4] = {0.f, 0.f, 0.f, 0.f}, up[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sidx = 0; sidx < nsplit; ++sidx) {
+      const float* src = p.part + (static_cast<int64_t>(u * nsplit + sidx) * kSplitRows + r) * 256;
+      const float4 a = *reinterpret_cast<const float4*>(src + 4 * lane);
+      const float4 c = *reinterpret_cast<const float4*>(src + 128 + 4 * lane);
+      g[0] += a.x; g[1] += a.y; g[2] += a.z; g[3] += a.w;
+      up[0] += c.x; up[1] += c.y; up[2] += c.z; up[3] += c.w;
+    }
+    float a[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = silu_f32(g[i]) * up[i];
+    const int64_t row = static_cast<int64_t>(b) * p.bm + r;
+    const int icol = j * kTI + 4 * lane;
+    if (kFp8) {
+      float amax = fmaxf(fmaxf(fabsf(a[0]), fabsf(a[1])), fmaxf(fabsf(a[2]), fabsf(a[3])));
+#pragma unroll
+      for (int d = 1; d < 8; d <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+      int sc = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127 - 8;
+      sc = sc < -127 ? -127 : (sc > 127 ? 127 : sc);
+      const float inv = __uint_as_float(static_cast<uint32_t>(127 - sc) << 23);
+      const uint32_t wv = static_cast<uint32_t>(cvt_e4m3x2(a[0] * inv, a[1] * inv)) |
+                          (static_cast<uint32_t>(cvt_e4m3x2(a[2] * inv, a[3] * inv)) << 16);
+      *reinterpret_cast<uint32_t*>(p.act + row * p.I + icol) = wv;
+      if ((lane & 7) == 0)
+        p.act_sf[(static_cast<int64_t>(b) * p.n_jt + j) * kSfTileBytes + (r & 31) * 16 + (r >> 5) * 4 + (lane >> 3)] =
+            static_cast<uint8_t>(sc + 127);
+    } else if (icol < p.I) {
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.act) + row * p.I + icol;
+      if (icol + 4 <= p.I) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (icol + i < p.I) dst[i] = __float2bfloat16_rn(a[i]);
+      }
+    }
   }
 }
 
@@ -845,7 +977,7 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const TP* __restrict__
 // host side
 // ========================================================================
 struct WsLayout {
-  int64_t act, act_sf, yw, flags, total;
+  int64_t act, act_sf, yw, flags, part, total;
   int64_t cap_rows;
 };
 
@@ -865,7 +997,9 @@ static WsLayout ws_layout(bool fp8, int T, int K, int N, int E, int top_k, int b
   w.yw = off;
   off = round_up(off + R * K * (fp8 ? 2 : 4), 1024);
   w.flags = off;
-  off = round_up(off + R * 4, 256);
+  off = round_up(off + R * 4, 1024);
+  w.part = off;
+  off = round_up(off + static_cast<int64_t>(kMaxSplitItems) * kSplitRows * 256 * 4, 256);
   w.total = off;
   return w;
 }
@@ -1025,6 +1159,7 @@ static int run_fused(const FusedArgs& a) {
   p1.act = ws + L.act;
   p1.act_sf = ws + L.act_sf;
   p1.flags = reinterpret_cast<int32_t*>(ws + L.flags);
+  p1.part = reinterpret_cast<float*>(ws + L.part);
   p1.status = status_ptr[dev];
   p1.K = a.K; p1.N = a.N; p1.I = I; p1.E = a.E; p1.top_k = a.top_k; p1.bm = a.bm;
   p1.R = a.T * a.top_k;
@@ -1061,7 +1196,9 @@ static int run_fused(const FusedArgs& a) {
   const int64_t units1 = static_cast<int64_t>(max_blocks) * p1.n_jt;
   const int64_t units2 = static_cast<int64_t>(max_blocks) * p2.n_ht;
   int ctas = req_ctas > 0 ? req_ctas : nsm;
-  const int grid1 = static_cast<int>(units1 < ctas ? units1 : ctas);
+  // one CTA per SM: small problems split their units' K range over the CTAs
+  const int grid1 = ctas;
+  (void)units1;
   const int grid2 = static_cast<int>(units2 < ctas ? units2 : ctas);
   // Each CTA allocates all 512 TMEM columns: request more than half of the
   // shared memory so that two CTAs never share an SM.
@@ -1104,6 +1241,10 @@ static int run_fused(const FusedArgs& a) {
   cudaError_t err = a.fp8 ? cudaLaunchKernelEx(&c1, moe_p1_kernel<true>, tm_w1, p1)
                           : cudaLaunchKernelEx(&c1, moe_p1_kernel<false>, tm_w1, p1);
   if (err != cudaSuccess) return cuda_fail("fused_moe: gate/up phase launch", err);
+  cudaLaunchConfig_t cr = config(nsm, 256, 0);
+  err = a.fp8 ? cudaLaunchKernelEx(&cr, moe_p1_reduce_kernel<true>, p1, grid1)
+              : cudaLaunchKernelEx(&cr, moe_p1_reduce_kernel<false>, p1, grid1);
+  if (err != cudaSuccess) return cuda_fail("fused_moe: split-K reduction launch", err);
   if ((rc = mark(1)) != MOE_OK) return rc;
   cudaLaunchConfig_t c2 = config(grid2, kP2Threads, smem2);
   err = a.fp8 ? cudaLaunchKernelEx(&c2, moe_p2_kernel<true>, tm_w2, tm_act, p2)

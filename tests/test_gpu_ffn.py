@@ -77,12 +77,15 @@ SMALL_BF16 = [
     small("bf16", 50, 384, 80, 6, 2, 16),         # I = 40: partial 64-wide K chunk in the down GEMM
     small("bf16", 300, 256, 256, 16, 4, 128, 1.2),  # skewed routing, empty experts
     small("bf16", 1, 128, 256, 4, 1, 128),
+    small("bf16", 12, 1024, 512, 4, 2, 64),       # few units, few rows: split-K (8 splits)
+    small("bf16", 10, 512, 320, 3, 2, 32),        # split-K with a partial intermediate tile (I = 160)
 ]
 SMALL_MXFP8 = [
     small("mxfp8", 200, 256, 512, 8, 2, 128),
     small("mxfp8", 200, 512, 256, 8, 2, 64),
     small("mxfp8", 90, 256, 768, 6, 3, 32),       # I = 384: 3 intermediate tiles
     small("mxfp8", 300, 256, 256, 16, 4, 128, 1.2),
+    small("mxfp8", 12, 1024, 512, 4, 2, 128),     # split-K (4 splits)
 ]
 
 
@@ -96,8 +99,9 @@ def test_small_full_oracle(sh):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "mxfp8"])
-def test_deterministic(dtype):
-    sh = small(dtype, 300, 256, 512, 8, 3, 128)
+@pytest.mark.parametrize("T", [300, 12])  # 12 tokens: the split-K path
+def test_deterministic(dtype, T):
+    sh = small(dtype, T, 1024 if T < 100 else 256, 512, 8, 3, 128)
     a, b = gpu_forward(sh, W.inputs(sh, seed=3), repeat=2)
     np.testing.assert_array_equal(a, b)
 
