@@ -431,7 +431,7 @@ def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
     l2 = ("L2 flushed between steps (512 MB written then read back, outside the per-step events)" if flush_l2 else
           f"inputs larger than L2 (touched expert weights {cm['bytes_w'] / 1e9:.2f} GB per step)")
     return {
-        "metric": METRIC, "value": world * cm["flops"] / (ms_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "metric": METRIC, "value": whole_job_tflops(cm["flops"], world, ms_step), "unit": "TFLOP/s",
         "n_gpus": world, "steps": steps, "warmup": warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": sh.dtype,
         "data": "synthetic (seeded workloads generator, random weights)",
@@ -450,6 +450,23 @@ def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
         "gpu_launches": m["launches"],
         "clocks": m["clocks"],
     }
+
+
+def max_over_ranks(v: float, world: int, dist=None, device=None) -> float:
+    """The maximum of a per-rank value over all ranks (every rank gets it)."""
+    if world == 1:
+        return v
+    import torch
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Replicas: every rank does the same work per step; the job's rate is the
+    sum of the ranks' work over the slowest rank's step time."""
+    return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
 def run_b200(args):
@@ -476,19 +493,12 @@ def run_b200(args):
     flush = args.flush_l2 or cm["bytes_w"] < 4 * 126e6
     m = measure(prob, args.steps, args.warmup, flush_l2=flush, barrier=barrier, local=local)
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    m["ms_step"] = max_over_ranks(m["ms_step"])
+    m["ms_step"] = max_over_ranks(m["ms_step"], world, dist, dev)
     line = result_line(sh, cm, m, world, args.steps, args.warmup, peaks, peak_src, flush)
     if not args.no_e2e:
         ems, h2d, d2h = measure_e2e(prob, args.steps, barrier)
-        ems = max_over_ranks(ems)
-        line["e2e"] = {"value": world * cm["flops"] / (ems / args.steps * 1e-3) / 1e12, "unit": "TFLOP/s",
+        ems = max_over_ranks(ems, world, dist, dev)
+        line["e2e"] = {"value": whole_job_tflops(cm["flops"], world, ems / args.steps), "unit": "TFLOP/s",
                        "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                        "us_per_call": 1e3 * ems / args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
