@@ -205,7 +205,9 @@ __device__ __forceinline__ int pf_id(const BlockPf& f, int q) {
 }
 
 // Number of K-splits per gate/up unit (1: no split), identical in every CTA
-// and in the reduction kernel.
+// and in the reduction kernel.  Splitting is used only while at least two
+// CTAs per unit would otherwise sit idle; more concurrent streams of smaller
+// K ranges measured slower on the weight stream than fewer longer ones.
 __device__ __forceinline__ int split_count(int n_units, int grid, int n_kc) {
   if (n_units <= 0 || 2 * n_units > grid) return 1;
   int sk = min(min(grid, kMaxSplitItems) / n_units, kMaxSplit);
@@ -510,6 +512,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       const bool mine = row_valid(bi, r);
       const int64_t row = static_cast<int64_t>(b) * p.bm + r;
       const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 256u;
+      bool released = false;
       if (nsplit > 1 && bi.nend <= kSplitRows) {
         // split item: hand the raw gate/up partials (rows < 32, quadrant 0)
         // to the reduction kernel
@@ -530,7 +533,50 @@ __global__ void __launch_bounds__(kP1Threads, 1)
             }
           }
         }
-      } else if (32 * q < bi.nend) {  // warp-uniform: skip quadrants with no routed row
+      } else if (32 * q < bi.nend && kFp8) {
+        // One TMEM accumulator on this path: the thread's whole slice (64
+        // intermediate columns of row r) is converted in registers and the
+        // accumulator handed back to the MMA warp before the global stores.
+        uint32_t wq[2][8];
+        int scq[2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int col0 = 64 * h + 32 * c;  // within the unit's 128-column tile
+          uint32_t gr[32], ur[32];
+          tmem_ld32(tacc + col0, gr);
+          tmem_ld32(tacc + 128 + col0, ur);
+          tmem_ld_wait();
+          float a[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = silu_f32(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(a[i]));
+          int sc = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127 - 8;
+          sc = sc < -127 ? -127 : (sc > 127 ? 127 : sc);
+          const float inv = __uint_as_float(static_cast<uint32_t>(127 - sc) << 23);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            wq[c][i] = static_cast<uint32_t>(cvt_e4m3x2(a[4 * i] * inv, a[4 * i + 1] * inv)) |
+                       (static_cast<uint32_t>(cvt_e4m3x2(a[4 * i + 2] * inv, a[4 * i + 3] * inv)) << 16);
+          scq[c] = sc;
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        released = true;
+        if (mine) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int col0 = 64 * h + 32 * c;
+            uint4* dst = reinterpret_cast<uint4*>(p.act + row * p.I + j * kTI + col0);
+            dst[0] = make_uint4(wq[c][0], wq[c][1], wq[c][2], wq[c][3]);
+            dst[1] = make_uint4(wq[c][4], wq[c][5], wq[c][6], wq[c][7]);
+            p.act_sf[(static_cast<int64_t>(b) * n_jt + j) * kSfTileBytes + (r & 31) * 16 + (r >> 5) * 4 +
+                     (col0 >> 5)] = static_cast<uint8_t>(scq[c] + 127);
+          }
+        }
+      } else if (32 * q < bi.nend) {  // bf16 (two accumulators: the stores overlap the next unit's MMAs)
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
           const int col0 = 64 * h + 32 * c;  // within the unit's 128-column tile
@@ -542,26 +588,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) a[i] = silu_f32(__uint_as_float(gr[i])) * __uint_as_float(ur[i]);
           const int icol = j * kTI + col0;
-          if (kFp8) {
-            float amax = 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(a[i]));
-            int sc = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127 - 8;
-            sc = sc < -127 ? -127 : (sc > 127 ? 127 : sc);
-            const float inv = __uint_as_float(static_cast<uint32_t>(127 - sc) << 23);
-            uint32_t w[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              w[i] = static_cast<uint32_t>(cvt_e4m3x2(a[4 * i] * inv, a[4 * i + 1] * inv)) |
-                     (static_cast<uint32_t>(cvt_e4m3x2(a[4 * i + 2] * inv, a[4 * i + 3] * inv)) << 16);
-            if (mine) {
-              uint4* dst = reinterpret_cast<uint4*>(p.act + row * p.I + icol);
-              dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-              dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-              p.act_sf[(static_cast<int64_t>(b) * n_jt + j) * kSfTileBytes + (r & 31) * 16 + (r >> 5) * 4 +
-                       (col0 >> 5)] = static_cast<uint8_t>(sc + 127);
-            }
-          } else if (mine && icol < p.I) {
+          if (mine && icol < p.I) {
             __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.act) + row * p.I + icol;
             if (icol + 32 <= p.I) {
               uint32_t w[16];
@@ -578,9 +605,11 @@ __global__ void __launch_bounds__(kP1Threads, 1)
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      }
       ++acc_it;
     }
   }
@@ -842,7 +871,54 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 256u;
-      if (32 * q < bi.nend) {
+      bool released = false;
+      if (32 * q < bi.nend && kFp8) {
+        // One TMEM accumulator on this path: the thread's weighted half-row is
+        // packed to bf16 in registers (up to 4 slices of 32 features) and the
+        // accumulator handed back to the MMA warp before the slices go through
+        // the staging buffer to global memory, as below.
+        const int half = nn / 2;
+        const int64_t col_base = static_cast<int64_t>(ht) * TH + h * half;
+        uint32_t pk[4][16];
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl) {
+          if (32 * sl < half) {  // uniform
+            uint32_t yr[32];
+            tmem_ld32(tacc + h * half + 32 * sl, yr);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[sl][i] = pack_bf16x2(wgt * __uint_as_float(yr[2 * i]), wgt * __uint_as_float(yr[2 * i + 1]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        released = true;
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl) {
+          if (32 * sl < half) {
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              stg4[lane * 4 + (i ^ ((lane >> 1) & 3))] =
+                  make_uint4(pk[sl][4 * i], pk[sl][4 * i + 1], pk[sl][4 * i + 2], pk[sl][4 * i + 3]);
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+              const int rl = 8 * it + (lane >> 2), cq = lane & 3;
+              const uint4 v = stg4[rl * 4 + (cq ^ ((rl >> 1) & 3))];
+              const int route_l = __shfl_sync(0xffffffffu, route, rl);
+              const int mine_l = __shfl_sync(0xffffffffu, static_cast<int>(mine), rl);
+              if (mine_l) {
+                const int64_t e0 = static_cast<int64_t>(route_l) * p.K + col_base + 32 * sl;
+                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.yw) + e0 + 8 * cq) = v;
+              }
+            }
+          }
+        }
+        if (mine && ht == 0 && h == 0) p.flags[route] = 1;
+      } else if (32 * q < bi.nend) {
         // Thread = row.  Each slice of the warp's 32 rows goes through shared
         // memory so that the stores leave as 64 contiguous bytes per row (8
         // rows per instruction) instead of 16 bytes to 32 different rows.
@@ -898,9 +974,11 @@ __global__ void __launch_bounds__(kP2Threads, 1)
         }
         if (mine && ht == 0 && h == 0) p.flags[route] = 1;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      }
       ++acc_it;
     }
   }
@@ -917,18 +995,38 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 // ========================================================================
 // combine: out[t] = bf16( sum_j yw[t*top_k + j] ), routes in order
 // ========================================================================
-__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+// 8 consecutive partials of one route, kept packed in registers until they
+// are summed (bf16: one 16-byte load, fp32: two), so that a thread holds all
+// of its routes' loads in flight with few registers.
+template <typename TP>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 a;
+};
+template <>
+struct Raw8<float> {
+  uint4 a, b;
+};
+__device__ __forceinline__ void load_raw8(const __nv_bfloat16* p, Raw8<__nv_bfloat16>& r) {
+  r.a = __ldg(reinterpret_cast<const uint4*>(p));
 }
-__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
-  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
-  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+__device__ __forceinline__ void load_raw8(const float* p, Raw8<float>& r) {
+  r.a = __ldg(reinterpret_cast<const uint4*>(p));
+  r.b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+}
+__device__ __forceinline__ void add_raw8(const Raw8<__nv_bfloat16>& r, float (&acc)[8]) {
+  const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    acc[2 * i] += __uint_as_float(w[i] << 16);
+    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
   }
+}
+__device__ __forceinline__ void add_raw8(const Raw8<float>& r, float (&acc)[8]) {
+  const uint32_t w[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] += __uint_as_float(w[i]);
 }
 
 // One thread sums 8 consecutive features of one token over its top_k routes.
@@ -937,7 +1035,7 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
 // then discarded), so a thread has all its loads in flight at once; the sum
 // runs in route order, so the result does not depend on scheduling.
 template <typename TP, int kMaxK>
-__global__ void __launch_bounds__(256) moe_combine_kernel(const TP* __restrict__ yw, const int32_t* __restrict__ flags,
+__global__ void __launch_bounds__(256, sizeof(TP) == 2 ? 4 : 2) moe_combine_kernel(const TP* __restrict__ yw, const int32_t* __restrict__ flags,
                                                           __nv_bfloat16* __restrict__ out, int T, int K, int top_k) {
   pdl_wait();  // the down phase's partial rows are read below
   const int kv = K / 8;
@@ -949,22 +1047,19 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const TP* __restrict__
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j0 = 0; j0 < top_k; j0 += kMaxK) {
       int f[kMaxK];
-      float y[kMaxK][8];
+      Raw8<TP> y[kMaxK];
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j) {
         f[j] = 0;
         if (j0 + j < top_k) {
           const int64_t r = t * top_k + j0 + j;
           f[j] = __ldg(flags + r);
-          load8(yw + r * K + h, y[j]);
+          load_raw8(yw + r * K + h, y[j]);
         }
       }
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j)
-        if (f[j]) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] += y[j][i];
-        }
+        if (f[j]) add_raw8(y[j], acc);
     }
     __nv_bfloat162 o[4];
 #pragma unroll
@@ -999,7 +1094,12 @@ static WsLayout ws_layout(bool fp8, int T, int K, int N, int E, int top_k, int b
   w.flags = off;
   off = round_up(off + R * 4, 1024);
   w.part = off;
-  off = round_up(off + static_cast<int64_t>(kMaxSplitItems) * kSplitRows * 256 * 4, 256);
+  {
+    // split items never exceed kMaxSplitItems nor kMaxSplit per possible unit
+    const int64_t max_units = (w.cap_rows / bm) * ((I + kTI - 1) / kTI);
+    const int64_t items = std::min<int64_t>(kMaxSplitItems, max_units * kMaxSplit);
+    off = round_up(off + items * kSplitRows * 256 * 4, 256);
+  }
   w.total = off;
   return w;
 }
@@ -1251,9 +1351,20 @@ static int run_fused(const FusedArgs& a) {
               : cudaLaunchKernelEx(&c2, moe_p2_kernel<false>, tm_w2, tm_act, p2);
   if (err != cudaSuccess) return cuda_fail("fused_moe: down phase launch", err);
   if ((rc = mark(2)) != MOE_OK) return rc;
+  // one full wave of resident blocks (grid-stride beyond it)
+  static int comb_occ[2] = {0, 0};
+  int& occ = comb_occ[a.fp8 ? 1 : 0];
+  if (occ == 0) {
+    int nb = 0;
+    err = a.fp8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<__nv_bfloat16, 8>, 256, 0)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<float, 8>, 256, 0);
+    if (err != cudaSuccess) return cuda_fail("fused_moe: combine occupancy query", err);
+    occ = nb < 1 ? 1 : nb;
+  }
   const int64_t nvec = static_cast<int64_t>(a.T) * (a.K / 8);
   const int64_t cblocks = (nvec + 255) / 256;
-  const int cgrid = static_cast<int>(cblocks < 8L * nsm ? cblocks : 8L * nsm);
+  const int64_t wave = static_cast<int64_t>(occ) * nsm;
+  const int cgrid = static_cast<int>(cblocks < wave ? cblocks : wave);
   cudaLaunchConfig_t c3 = config(cgrid, 256, 0);
   __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(a.out);
   err = a.fp8 ? cudaLaunchKernelEx(&c3, moe_combine_kernel<__nv_bfloat16, 8>,
