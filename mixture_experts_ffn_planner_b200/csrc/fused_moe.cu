@@ -121,6 +121,7 @@ struct P2Params {
   int w_reuse;
   int n_ht;                 // ceil(K / 256): work units per planner block
   int n_kc;                 // K-chunks of the down GEMM
+  int a_full;               // the stage's A region holds 128 rows
   int stages, stage_bytes;
   int off_b, off_sf;
 };
@@ -692,7 +693,8 @@ __global__ void __launch_bounds__(256) moe_p1_reduce_kernel(const __grid_constan
 // ========================================================================
 template <bool kFp8>
 __global__ void __launch_bounds__(kP2Threads, 1)
-    moe_p2_kernel(const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_act,
+    moe_p2_kernel(const __grid_constant__ CUtensorMap tm_w2, const __grid_constant__ CUtensorMap tm_w2x,
+                  const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_actx,
                   const __grid_constant__ P2Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -720,7 +722,9 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_w2);
+    prefetch_tmap(&tm_w2x);
     prefetch_tmap(&tm_act);
+    prefetch_tmap(&tm_actx);
   }
   if (warp == 1) {
     tmem_alloc(tmem_base_sm, 512);
@@ -756,17 +760,29 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       if (bi.nend == 0) continue;
       const int nb = min(TH, p.K - ht * TH) / 128;  // 128-row pieces of this feature tile
       const int w2_row = bi.e * p.K + ht * TH;
-      const uint32_t tx = nb * 128 * kRowBytes + bi.n16 * kRowBytes + (kFp8 ? (1 + nb) * kSfTileBytes : 0);
+      // A block of at least 64 rows takes its intermediate rows as one
+      // 128-row box (rows past the block are loaded and never stored) and a
+      // full feature tile its w2 rows as one 256-row box: fewer, larger copies
+      // per stage than 16-row and 128-row pieces.
+      const bool big_a = p.a_full && bi.n16 >= 64;
+      const int a_rows = big_a ? 128 : bi.n16;
+      const uint32_t tx = nb * 128 * kRowBytes + a_rows * kRowBytes + (kFp8 ? (1 + nb) * kSfTileBytes : 0);
       for (int kc = 0; kc < p.n_kc; ++kc) {
         if (lane == 0) {
           ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
           if (ok) {
             uint8_t* st = stage_ptr(s);
             mbar_arrive_expect_tx(&full[s], tx);
-            for (int i = 0; i < bi.n16 / 16; ++i)
-              tma_load_2d(st + i * 16 * kRowBytes, &tm_act, &full[s], kc * kKC, b * p.bm + 16 * i, pol_a);
-            for (int i = 0; i < nb; ++i)
-              tma_load_2d(st + p.off_b + i * 128 * kRowBytes, &tm_w2, &full[s], kc * kKC, w2_row + 128 * i, pol_w);
+            if (big_a) {
+              tma_load_2d(st, &tm_actx, &full[s], kc * kKC, b * p.bm, pol_a);
+            } else {
+              for (int i = 0; i < bi.n16 / 16; ++i)
+                tma_load_2d(st + i * 16 * kRowBytes, &tm_act, &full[s], kc * kKC, b * p.bm + 16 * i, pol_a);
+            }
+            if (nb == 2)
+              tma_load_2d(st + p.off_b, &tm_w2x, &full[s], kc * kKC, w2_row, pol_w);
+            else
+              tma_load_2d(st + p.off_b, &tm_w2, &full[s], kc * kKC, w2_row, pol_w);
             if (kFp8) {
               bulk_load(st + p.off_sf, p.act_sf + (static_cast<int64_t>(b) * KT2 + kc) * kSfTileBytes, kSfTileBytes,
                         &full[s]);
@@ -1235,11 +1251,19 @@ static int run_fused(const FusedArgs& a) {
     status_ptr[dev] = static_cast<int*>(sp);
   }
 
-  CUtensorMap tm_w1, tm_w2, tm_act;
+  CUtensorMap tm_w1, tm_w2, tm_w2x, tm_act, tm_actx;
   int rc;
   if ((rc = make_tmap(&tm_w1, a.w1, a.fp8, static_cast<int64_t>(a.E) * a.N, a.K, 128)) != MOE_OK) return rc;
   if ((rc = make_tmap(&tm_w2, a.w2, a.fp8, static_cast<int64_t>(a.E) * a.K, I, 128)) != MOE_OK) return rc;
   if ((rc = make_tmap(&tm_act, ws + L.act, a.fp8, L.cap_rows, I, 16)) != MOE_OK) return rc;
+  // the one-box forms are encoded only where the down phase can use them
+  // (full 256-feature tiles; 128-row A regions)
+  tm_w2x = tm_w2;
+  tm_actx = tm_act;
+  const int a_rows = a_region_rows(a.bm, static_cast<int64_t>(a.T) * a.top_k);
+  if (a.K >= 2 * 128 && (rc = make_tmap(&tm_w2x, a.w2, a.fp8, static_cast<int64_t>(a.E) * a.K, I, 256)) != MOE_OK)
+    return rc;
+  if (a_rows >= kM && (rc = make_tmap(&tm_actx, ws + L.act, a.fp8, L.cap_rows, I, 128)) != MOE_OK) return rc;
 
   const int nsm = sm_count();
   if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(SM count)");
@@ -1266,7 +1290,6 @@ static int run_fused(const FusedArgs& a) {
   p1.max_blocks = max_blocks;
   p1.w_reuse = static_cast<int64_t>(a.T) * a.top_k >= static_cast<int64_t>(a.E) * a.bm ? 1 : 0;
   p1.n_jt = (I + kTI - 1) / kTI;
-  const int a_rows = a_region_rows(a.bm, static_cast<int64_t>(a.T) * a.top_k);
   p1.stage_bytes = stage_bytes(a.fp8, a_rows);
   p1.off_b = off_b_of(a_rows);
   p1.off_sf = off_sf_of(a_rows);
@@ -1289,6 +1312,7 @@ static int run_fused(const FusedArgs& a) {
   p2.n_kc = a.fp8 ? I / 128 : (I + 63) / 64;
   p2.stage_bytes = stage_bytes(a.fp8, a_rows);
   p2.off_b = p1.off_b;
+  p2.a_full = a_rows >= kM ? 1 : 0;
   p2.off_sf = p1.off_sf;
   p2.stages = pick_stages(p2.stage_bytes, kP2Ctrl + kP2Staging, req_stages, 8);
   if (p1.stages < 2 || p2.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "%s: shared memory too small", nm);
@@ -1347,8 +1371,8 @@ static int run_fused(const FusedArgs& a) {
   if (err != cudaSuccess) return cuda_fail("fused_moe: split-K reduction launch", err);
   if ((rc = mark(1)) != MOE_OK) return rc;
   cudaLaunchConfig_t c2 = config(grid2, kP2Threads, smem2);
-  err = a.fp8 ? cudaLaunchKernelEx(&c2, moe_p2_kernel<true>, tm_w2, tm_act, p2)
-              : cudaLaunchKernelEx(&c2, moe_p2_kernel<false>, tm_w2, tm_act, p2);
+  err = a.fp8 ? cudaLaunchKernelEx(&c2, moe_p2_kernel<true>, tm_w2, tm_w2x, tm_act, tm_actx, p2)
+              : cudaLaunchKernelEx(&c2, moe_p2_kernel<false>, tm_w2, tm_w2x, tm_act, tm_actx, p2);
   if (err != cudaSuccess) return cuda_fail("fused_moe: down phase launch", err);
   if ((rc = mark(2)) != MOE_OK) return rc;
   // one full wave of resident blocks (grid-stride beyond it)
