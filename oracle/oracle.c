@@ -188,6 +188,61 @@ int orc_moe_align(const int32_t* topk_ids, int T, int top_k, int E, int block_m,
 }
 
 /* ====================================================================== */
+/* Router ahead of the planner.  "Prime Flash MoE", Usage: topk_ids come  */
+/* from the caller's gate; "[RFC] Fused W8A8 MoE megakernel on H20",      */
+/* Results so far: both paths run with the same normalized routing        */
+/* weights.  Reading taken (the plainest one those two support): a        */
+/* softmax over the experts of a per-expert score, the top_k largest kept */
+/* and their probabilities renormalised to sum to one.                    */
+/*  - score z[t][e] = logits[t][e] + bias[e], formed in fp32: the scores  */
+/*    decide integer ids, so the decision is taken in the precision the   */
+/*    device forms them in;                                               */
+/*  - experts ranked by descending z, equal scores by ascending index;    */
+/*  - weight of kept expert j = exp(z_j) / sum over kept i of exp(z_i),   */
+/*    in double (the full softmax denominator cancels in the              */
+/*    renormalisation), evaluated as exp(z_j - z_max) for range.          */
+/* Scores must be finite.                                                 */
+/* ====================================================================== */
+
+int orc_route_topk(const float* logits, const float* bias, int T, int E, int top_k,
+                   int32_t* topk_ids, double* topk_weights) {
+  if (T < 0 || E < 1 || top_k < 1 || top_k > E) return -1;
+  float* z = (float*)malloc((size_t)E * sizeof(float));
+  unsigned char* taken = (unsigned char*)malloc((size_t)E);
+  if (!z || !taken) { free(z); free(taken); return -1; }
+  for (int t = 0; t < T; ++t) {
+    for (int e = 0; e < E; ++e) {
+      const float b = bias ? bias[e] : 0.0f;
+      z[e] = logits[(int64_t)t * E + e] + b; /* one fp32 addition */
+      taken[e] = 0;
+    }
+    int32_t* ids = topk_ids + (int64_t)t * top_k;
+    double* w = topk_weights + (int64_t)t * top_k;
+    /* selection: repeatedly the largest remaining score, lowest index first */
+    for (int j = 0; j < top_k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e) {
+        if (taken[e]) continue;
+        if (best < 0 || z[e] > z[best]) best = e;
+      }
+      taken[best] = 1;
+      ids[j] = best;
+    }
+    /* renormalised softmax over the kept experts */
+    const double zmax = (double)z[ids[0]];
+    double sum = 0.0;
+    for (int j = 0; j < top_k; ++j) {
+      w[j] = exp((double)z[ids[j]] - zmax);
+      sum += w[j];
+    }
+    for (int j = 0; j < top_k; ++j) w[j] /= sum;
+  }
+  free(z);
+  free(taken);
+  return 0;
+}
+
+/* ====================================================================== */
 /* [PFM] Scale layout (mxfp8): weight scales reordered into a sequence of */
 /* 512-byte tiles, each covering 128 MN x 128 K (= 4 scale bytes along K). */
 /* Tile order: expert, then MN tile, then K tile.  Inside a tile row r and */

@@ -39,6 +39,12 @@ int orc_moe_align(const int32_t* topk_ids, int T, int top_k, int E, int block_m,
                   int32_t* sorted_token_ids, int32_t* expert_ids,
                   int32_t* num_tokens_post_padded, int64_t capacity);
 
+/* ---- router (softmax, top-k, renormalisation) -------------------------- */
+/* bias may be NULL.  ids ranked by descending fp32 score logits+bias (ties:
+ * lower index); weights in double.  Returns 0, or -1 on bad sizes. */
+int orc_route_topk(const float* logits, const float* bias, int T, int E, int top_k,
+                   int32_t* topk_ids, double* topk_weights);
+
 /* ---- blocked weight-scale layout --------------------------------------- */
 int64_t orc_pack_scales_bytes(int E, int MN, int KS);
 void orc_pack_scales_blocked(const uint8_t* in, uint8_t* out, int E, int MN, int KS);
