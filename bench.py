@@ -60,6 +60,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--router", action="store_true",
+                    help="start each step from router logits (moe_route_align) instead of routed ids")
     ap.add_argument("--stages", type=int, default=0)
     ap.add_argument("--ctas", type=int, default=0)
     ap.add_argument("--flush-l2", action="store_true",
@@ -248,7 +250,7 @@ def run_reference(args):
 class Problem:
     """Device-resident inputs of one workload and one step of the hot path."""
 
-    def __init__(self, sh: W.Shape, inp: dict, dev, stages: int = 0, ctas: int = 0):
+    def __init__(self, sh: W.Shape, inp: dict, dev, stages: int = 0, ctas: int = 0, router: bool = False):
         import torch
 
         import mixture_experts_ffn_planner_b200 as moe
@@ -260,7 +262,15 @@ class Problem:
             return (t.view(dtype) if dtype is not None else t).to(dev)
 
         bm = self.bm = sh.block_m
-        self.ids, self.tw = up(inp["topk_ids"]), up(inp["topk_weights"])
+        self.router = router
+        if router:
+            # the step starts from router logits: moe_route_align writes ids and weights
+            self.logits = up(inp["router_logits"])
+            self.bias = None if inp["router_bias"] is None else up(inp["router_bias"])
+            self.ids = torch.empty((sh.T, sh.top_k), dtype=torch.int32, device=dev)
+            self.tw = torch.empty((sh.T, sh.top_k), dtype=torch.float32, device=dev)
+        else:
+            self.ids, self.tw = up(inp["topk_ids"]), up(inp["topk_weights"])
         cap = moe.moe_align_capacity(sh.T, sh.top_k, sh.E, bm)
         self.s_ids = torch.empty(cap, dtype=torch.int32, device=dev)
         self.e_ids = torch.empty((cap + bm - 1) // bm, dtype=torch.int32, device=dev)
@@ -280,7 +290,9 @@ class Problem:
                               dtype=torch.uint8, device=dev)
         self.plain = moe.Tuning(stages, ctas, None)
         self.stages, self.ctas = stages, ctas
-        self.launches_per_step = 4  # moe_align, gate/up phase, down phase, reduction
+        # planner, gate/up phase, split-K reduction, down phase, combine (+ the router kernel for
+        # batches of more than 128 tokens on the router path)
+        self.launches_per_step = 5 + (1 if router and sh.T > 128 else 0)
 
     def fused(self, tune):
         m = self.moe
@@ -294,7 +306,11 @@ class Problem:
     def step(self, tune=None, plan_event=None):
         if plan_event is not None:
             plan_event.record()
-        self.moe.moe_align(self.ids, self.sh.E, self.bm, self.s_ids, self.e_ids, self.ntpp)
+        if self.router:
+            self.moe.moe_route_align(self.logits, self.sh.top_k, self.bm, self.bias, self.ids, self.tw, self.s_ids,
+                                     self.e_ids, self.ntpp)
+        else:
+            self.moe.moe_align(self.ids, self.sh.E, self.bm, self.s_ids, self.e_ids, self.ntpp)
         self.fused(self.plain if tune is None else tune)
 
 
@@ -382,9 +398,16 @@ def measure_e2e(prob: Problem, steps: int, barrier=None):
     stream = torch.cuda.current_stream()
     hx = torch.from_numpy(np.ascontiguousarray(inp["x"]))
     hx = hx.view(torch.bfloat16) if sh.dtype == "bf16" else hx
-    host_in = [hx.pin_memory(), torch.from_numpy(inp["topk_ids"]).pin_memory(),
-               torch.from_numpy(inp["topk_weights"]).pin_memory()]
-    dev_in = [prob.x, prob.ids, prob.tw]
+    if prob.router:
+        host_in = [hx.pin_memory(), torch.from_numpy(inp["router_logits"]).pin_memory()]
+        dev_in = [prob.x, prob.logits]
+        if prob.bias is not None:
+            host_in.append(torch.from_numpy(inp["router_bias"]).pin_memory())
+            dev_in.append(prob.bias)
+    else:
+        host_in = [hx.pin_memory(), torch.from_numpy(inp["topk_ids"]).pin_memory(),
+                   torch.from_numpy(inp["topk_weights"]).pin_memory()]
+        dev_in = [prob.x, prob.ids, prob.tw]
     if sh.dtype == "mxfp8":
         host_in.append(torch.from_numpy(np.ascontiguousarray(inp["x_scales"])).pin_memory())
         dev_in.append(prob.xs)
@@ -492,13 +515,17 @@ def run_b200(args):
 
     sh = W.shape(args.workload, args.tokens, **({"E": args.experts} if args.experts else {}))
     inp = W.inputs(sh, seed=args.seed + rank)  # every replica gets its own batch
+    if args.router:
+        inp["router_logits"], inp["router_bias"] = W.router_logits(sh, seed=args.seed + rank)
     cm = cost_model(sh, inp["topk_ids"], peaks)
-    prob = Problem(sh, inp, dev, args.stages, args.ctas)
+    prob = Problem(sh, inp, dev, args.stages, args.ctas, router=args.router)
     flush = args.flush_l2 or cm["bytes_w"] < 4 * 126e6
     m = measure(prob, args.steps, args.warmup, flush_l2=flush, barrier=barrier, local=local)
 
     m["ms_step"] = max_over_ranks(m["ms_step"], world, dist, dev)
     line = result_line(sh, cm, m, world, args.steps, args.warmup, peaks, peak_src, flush)
+    if args.router:
+        line["config"]["router"] = "in the step: moe_route_align (softmax, top-k, renormalise) from fp32 logits"
     if not args.no_e2e:
         ems, h2d, d2h = measure_e2e(prob, args.steps, barrier)
         ems = max_over_ranks(ems, world, dist, dev)

@@ -97,6 +97,32 @@ MOE_API int moe_align(const int32_t* topk_ids, int T, int top_k, int E, int bloc
               int64_t capacity, moe_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * moe_route_align -- the router fused ahead of the planner: softmax over the
+ * experts, top-k, renormalised weights, then exactly what moe_align does on
+ * the resulting ids.  [PFM] Usage: topk_ids come from the caller's gate;
+ * [RFC] Results so far: both paths use the same normalized routing weights.
+ * Reading: score z[t][e] = logits[t][e] + bias[e] formed in fp32; experts
+ * ranked by descending z, equal scores by ascending index; the first top_k
+ * kept, weight j = exp(z_j - z_0) / sum over the kept of exp(z_i - z_0).
+ *
+ *   logits              (T, E) fp32, device, row major, read only; finite.
+ *   bias                (E) fp32, device, or NULL for none.
+ *   topk_ids            (T, top_k) int32, device, written: kept experts in
+ *                       rank order.
+ *   topk_weights        (T, top_k) fp32, device, written; each row sums to 1.
+ *   sorted_token_ids, expert_ids, num_tokens_post_padded, capacity: as for
+ *                       moe_align (the same bits moe_align gives on topk_ids).
+ * Batches of at most 32 tokens are routed inside the planner's CTA; larger
+ * ones by an all-SM router kernel chained to the planner.
+ * Constraints: as moe_align, plus 1 <= top_k <= min(8, E).  Returns
+ * MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG before any launch otherwise.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_route_align(const float* logits, const float* bias, int T, int E, int top_k, int block_m,
+                    int32_t* topk_ids, float* topk_weights, int32_t* sorted_token_ids,
+                    int32_t* expert_ids, int32_t* num_tokens_post_padded, int64_t capacity,
+                    moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * pack_scales_blocked -- [PFM] Scale layout (mxfp8): weight scales (one e8m0
  * byte per 32 along K) reordered into a sequence of 512-byte tiles, each
  * covering 128 rows (MN) x 128 K (4 scale bytes).  Tile (e, mt, kt) starts at

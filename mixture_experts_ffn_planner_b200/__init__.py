@@ -11,6 +11,10 @@ Entry points (same names as the C ABI):
   padded to ``block_m``, and the row-to-token map ("[RFC] Fused W8A8 MoE
   megakernel on H20", Design; "Prime Flash MoE: Fused MoE Kernels for
   Blackwell", API / Shapes).
+* ``moe_route_align`` -- the router ahead of the planner: softmax over the
+  experts, top-k, renormalised weights, then the planner on the kept ids
+  ("Prime Flash MoE", Usage; "[RFC] Fused W8A8 MoE megakernel on H20",
+  Results so far).
 * ``fused_moe_bf16`` / ``fused_moe_mxfp8`` -- gather, gate/up GEMM, SwiGLU
   (mxfp8: on-chip requant of the intermediate), down GEMM and the top-k
   weighted reduction into ``out`` ("Prime Flash MoE", intro / API / Shapes).
@@ -26,7 +30,7 @@ import threading
 from . import _build
 
 __all__ = [
-    "MoeError", "load", "moe_align", "moe_align_capacity", "fused_moe_bf16", "fused_moe_mxfp8",
+    "MoeError", "load", "moe_align", "moe_align_capacity", "moe_route_align", "fused_moe_bf16", "fused_moe_mxfp8",
     "pack_scales_blocked", "pack_scales_blocked_bytes", "moe_workspace_bytes", "moe_device_status",
     "Tuning", "DTYPE_BF16", "DTYPE_MXFP8", "LIB_PATH", "fused_moe_bf16_noalloc",
     "fused_moe_bf16_noalloc_max_workspace",
@@ -77,6 +81,7 @@ _SIGS = {
     "moe_device_status": ([_P], _I),
     "moe_align_capacity": ([_I, _I, _I, _I], _I64),
     "moe_align": ([_P, _I, _I, _I, _I, _P, _P, _P, _I64, _P], _I),
+    "moe_route_align": ([_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I64, _P], _I),
     "pack_scales_blocked_bytes": ([_I, _I, _I], _I64),
     "pack_scales_blocked": ([_P, _P, _I, _I, _I, _P], _I),
     "moe_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I], _I64),
@@ -183,6 +188,48 @@ def moe_align(topk_ids, E: int, block_m: int, sorted_token_ids=None, expert_ids=
     _check(load().moe_align(_ptr(topk_ids), T, top_k, E, block_m, _ptr(sorted_token_ids), _ptr(expert_ids),
                             _ptr(num_tokens_post_padded), sorted_token_ids.numel(), _stream(stream)))
     return sorted_token_ids, expert_ids, num_tokens_post_padded
+
+
+def moe_route_align(logits, top_k: int, block_m: int, bias=None, topk_ids=None, topk_weights=None,
+                    sorted_token_ids=None, expert_ids=None, num_tokens_post_padded=None, stream=None):
+    """Router + planner.  logits (T, E) fp32, bias (E,) fp32 or None.  Returns (topk_ids,
+    topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded)."""
+    import torch
+
+    _need(logits, "logits", (torch.float32,))
+    T, E = logits.shape
+    if bias is not None:
+        _need(bias, "bias", (torch.float32,))
+        if bias.numel() != E:
+            raise ValueError("bias must hold E values")
+    cap = moe_align_capacity(T, top_k, E, block_m)
+    if cap < 0:
+        raise MoeError(-1, "moe_route_align: invalid sizes")
+    dev = logits.device
+    if topk_ids is None:
+        topk_ids = torch.empty((T, top_k), dtype=torch.int32, device=dev)
+    if topk_weights is None:
+        topk_weights = torch.empty((T, top_k), dtype=torch.float32, device=dev)
+    if sorted_token_ids is None:
+        sorted_token_ids = torch.empty(cap, dtype=torch.int32, device=dev)
+    if expert_ids is None:
+        expert_ids = torch.empty((sorted_token_ids.numel() + block_m - 1) // block_m, dtype=torch.int32,
+                                 device=dev)
+    if num_tokens_post_padded is None:
+        num_tokens_post_padded = torch.empty(1, dtype=torch.int32, device=dev)
+    _need(topk_ids, "topk_ids", (torch.int32,))
+    _need(topk_weights, "topk_weights", (torch.float32,))
+    if topk_ids.numel() < T * top_k or topk_weights.numel() < T * top_k:
+        raise ValueError("topk_ids / topk_weights must hold T * top_k entries")
+    for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
+                 (num_tokens_post_padded, "num_tokens_post_padded")):
+        _need(t, n, (torch.int32,))
+    if expert_ids.numel() < (sorted_token_ids.numel() + block_m - 1) // block_m:
+        raise ValueError("expert_ids must hold ceil(capacity / block_m) entries")
+    _check(load().moe_route_align(_ptr(logits), _ptr(bias), T, E, top_k, block_m, _ptr(topk_ids),
+                                  _ptr(topk_weights), _ptr(sorted_token_ids), _ptr(expert_ids),
+                                  _ptr(num_tokens_post_padded), sorted_token_ids.numel(), _stream(stream)))
+    return topk_ids, topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded
 
 
 def pack_scales_blocked(scales, out=None, stream=None):

@@ -32,6 +32,8 @@
 // Slots that receive no id (segment padding and the capacity tail) get -1,
 // and expert_ids is filled block by block; these writes are spread over the
 // cluster's CTAs.
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -73,10 +75,114 @@ __device__ __forceinline__ int32_t ld_dsmem(const int32_t* local, uint32_t rank)
   return v;
 }
 
+// ------------------------------------------------------------------ router
+// Softmax -> top-k -> renormalisation ahead of the planner.  "Prime Flash
+// MoE", Usage: topk_ids come from the caller's gate; "[RFC] Fused W8A8 MoE
+// megakernel on H20", Results so far: the paths share normalized routing
+// weights.  Reading: score z = logit + bias (fp32), experts ranked by
+// descending z with equal scores by ascending index, the first top_k kept,
+// weights = exp(z_j - z_0) / sum over the kept of exp(z_i - z_0) (the full
+// softmax denominator cancels in the renormalisation).  Scores must be finite.
+constexpr int kRouteMaxK = 8;
+// Batches of at most this many tokens (one per warp of the planner CTA) are
+// routed inside the planner; larger ones in their own all-SM kernel, which
+// measured faster from two tokens per warp on.
+constexpr int kRouteFusedMaxTokens = 32;
+
+// One warp routes token t.  Lane l scans experts l, l+32, ... keeping its
+// best kRouteMaxK in a sorted register list (compare-and-swap down a fixed
+// list, so equal scores keep the earlier, lower index ahead); k rounds of a
+// warp-wide arg-max (ties to the lower index) then merge the 32 lists.  Lane
+// j < k ends with the j-th expert and its weight, written to the outputs and,
+// when ids16 is given, to the staged id array at position t*k + j - id0.
+__device__ __forceinline__ void route_token(const float* __restrict__ logits, const float* __restrict__ bias,
+                                            int t, int E, int k, int lane, int32_t* __restrict__ topk_ids,
+                                            float* __restrict__ topk_w, uint16_t* ids16, int id0) {
+  float lv[kRouteMaxK];
+  int le[kRouteMaxK];
+#pragma unroll
+  for (int p = 0; p < kRouteMaxK; ++p) {
+    lv[p] = -INFINITY;
+    le[p] = 0x7fffffff;
+  }
+  const float* row = logits + static_cast<int64_t>(t) * E;
+  for (int e = lane; e < E; e += 32) {
+    float cv = __ldg(row + e) + (bias ? __ldg(bias + e) : 0.0f);
+    int ce = e;
+#pragma unroll
+    for (int p = 0; p < kRouteMaxK; ++p) {
+      if (cv > lv[p]) {
+        const float tv = lv[p];
+        const int te = le[p];
+        lv[p] = cv;
+        le[p] = ce;
+        cv = tv;
+        ce = te;
+      }
+    }
+  }
+  float my_v = 0.f;
+  int my_e = -1;
+  for (int j = 0; j < k; ++j) {
+    float bv = lv[0];
+    int be = le[0];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if (lane == j) {
+      my_v = bv;
+      my_e = be;
+    }
+    if (le[0] == be) {  // the owning lane drops its head
+#pragma unroll
+      for (int p = 0; p + 1 < kRouteMaxK; ++p) {
+        lv[p] = lv[p + 1];
+        le[p] = le[p + 1];
+      }
+      lv[kRouteMaxK - 1] = -INFINITY;
+      le[kRouteMaxK - 1] = 0x7fffffff;
+    }
+  }
+  const float z0 = __shfl_sync(0xffffffffu, my_v, 0);
+  float w = lane < k ? expf(my_v - z0) : 0.f;
+  float sum = w;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  if (lane < k) {
+    const int64_t r = static_cast<int64_t>(t) * k + lane;
+    topk_ids[r] = my_e;
+    topk_w[r] = w / sum;
+    if (ids16) ids16[r - id0] = static_cast<uint16_t>(my_e);
+  }
+}
+
+// Router for larger batches: one warp per token over the whole GPU; the
+// planner that follows is chained by programmatic dependent launch.
+__global__ void __launch_bounds__(256) moe_route_kernel(const float* __restrict__ logits,
+                                                        const float* __restrict__ bias, int T, int E, int k,
+                                                        int32_t* __restrict__ topk_ids,
+                                                        float* __restrict__ topk_w) {
+  pdl_launch_dependents();
+  const int lane = threadIdx.x & 31;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, nw = (gridDim.x * blockDim.x) >> 5;
+  for (int t = gw; t < T; t += nw) route_token(logits, bias, t, E, k, lane, topk_ids, topk_w, nullptr, 0);
+}
+
+// Planner.  With route_T > 0 (one CTA, at most one token per warp) the CTA first
+// routes route_T tokens itself from logits/bias, writing topk_ids/topk_w and
+// staging the ids directly; otherwise it reads topk_ids.
 __global__ void __launch_bounds__(kAlignThreads, 1)
     moe_align_kernel(const int32_t* __restrict__ topk_ids, int R, int E, int block_m,
                      int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids,
-                     int32_t* __restrict__ ntpp_out, int64_t capacity, int staged) {
+                     int32_t* __restrict__ ntpp_out, int64_t capacity, int staged,
+                     const float* __restrict__ logits, const float* __restrict__ bias, int route_T, int route_k,
+                     int32_t* route_ids, float* __restrict__ route_w) {
   extern __shared__ int32_t sm[];
   int32_t* hist = sm;                         // [kAlignWarps][E], later start offsets
   int32_t* cnt = hist + kAlignWarps * E;      // [E] this CTA's count per expert
@@ -86,6 +192,7 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
   uint16_t* ids16 = reinterpret_cast<uint16_t*>(warp_tot + kAlignWarps);  // [chunk] when staged
 
   pdl_launch_dependents();  // the fused phases may start their prologue now
+  pdl_wait();               // a preceding router kernel's ids (no-op after an ordinary launch)
   const uint32_t crank = cluster_ctarank(), csize = cluster_nctarank();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cchunk = (R + static_cast<int>(csize) - 1) / static_cast<int>(csize);
@@ -93,8 +200,12 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
 
   for (int i = tid; i < kAlignWarps * E; i += kAlignThreads) hist[i] = 0;
   // 0. stage this CTA's ids (independent loads, so their latencies overlap);
-  //    ids outside [0, E) route nowhere
-  if (staged) {
+  //    ids outside [0, E) route nowhere.  A routing CTA (one CTA, clo = 0)
+  //    produces them instead.
+  if (route_T > 0) {
+    for (int t = warp; t < route_T; t += kAlignWarps)
+      route_token(logits, bias, t, E, route_k, lane, route_ids, route_w, ids16, 0);
+  } else if (staged) {
 #pragma unroll 4
     for (int i = clo + tid; i < chi; i += kAlignThreads) {
       const int e = __ldg(topk_ids + i);
@@ -226,6 +337,54 @@ extern "C" int64_t moe_align_capacity(int T, int top_k, int E, int block_m) {
   return static_cast<int64_t>(T) * top_k + static_cast<int64_t>(E) * (block_m - 1);
 }
 
+// Launches the planner: one CTA, or one cluster of kAlignClusterMax CTAs for
+// large inputs.  route_T > 0 makes the (single) CTA route the tokens itself;
+// after_router chains the launch to a preceding router kernel.
+static int launch_align(const int32_t* topk_ids, int T, int top_k, int E, int block_m, int32_t* sorted_token_ids,
+                        int32_t* expert_ids, int32_t* num_tokens_post_padded, int64_t capacity, moe_stream_t stream,
+                        const float* logits, const float* bias, int route_T, int32_t* route_ids, float* route_w,
+                        bool after_router) {
+  const int R = T * top_k;
+  const int csize = R >= kAlignClusterMinIds ? kAlignClusterMax : 1;
+  const int cchunk = (R + csize - 1) / csize;
+  const size_t base = align_smem_base(E);
+  const size_t staged_bytes = base + sizeof(uint16_t) * static_cast<size_t>(cchunk);
+  const int staged = staged_bytes <= static_cast<size_t>(kAlignSmemLimit) ? 1 : 0;
+  const size_t smem = staged ? staged_bytes : base;
+  if (route_T > 0 && (csize != 1 || !staged))
+    return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: the in-planner router needs one CTA with staged ids");
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("moe_align: cudaGetDevice");
+  static bool attr_set[kMaxDevices] = {};
+  if (dev < kMaxDevices && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(moe_align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAlignSmemLimit) !=
+        cudaSuccess)
+      return cuda_fail("moe_align: cudaFuncSetAttribute");
+    attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(csize, 1, 1);
+  cfg.blockDim = dim3(kAlignThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_router ? 2 : 1;
+  const cudaError_t lerr = cudaLaunchKernelEx(&cfg, moe_align_kernel, topk_ids, R, E, block_m, sorted_token_ids,
+                                              expert_ids, num_tokens_post_padded, capacity, staged, logits, bias,
+                                              route_T, top_k, route_ids, route_w);
+  if (lerr != cudaSuccess) return cuda_fail("moe_align: launch", lerr);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return cuda_fail("moe_align: launch", err);
+  return MOE_OK;
+}
+
 extern "C" int moe_align(const int32_t* topk_ids, int T, int top_k, int E, int block_m,
                          int32_t* sorted_token_ids, int32_t* expert_ids, int32_t* num_tokens_post_padded,
                          int64_t capacity, moe_stream_t stream) {
@@ -244,38 +403,40 @@ extern "C" int moe_align(const int32_t* topk_ids, int T, int top_k, int E, int b
   if ((T > 0 && !topk_ids) || !sorted_token_ids || !expert_ids || !num_tokens_post_padded)
     return fail(MOE_ERR_INVALID_ARG, "moe_align: null pointer");
 
-  const int R = T * top_k;
-  const int csize = R >= kAlignClusterMinIds ? kAlignClusterMax : 1;
-  const int cchunk = (R + csize - 1) / csize;
-  const size_t base = align_smem_base(E);
-  const size_t staged_bytes = base + sizeof(uint16_t) * static_cast<size_t>(cchunk);
-  const int staged = staged_bytes <= static_cast<size_t>(kAlignSmemLimit) ? 1 : 0;
-  const size_t smem = staged ? staged_bytes : base;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("moe_align: cudaGetDevice");
-  static bool attr_set[kMaxDevices] = {};
-  if (dev < kMaxDevices && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(moe_align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAlignSmemLimit) !=
-        cudaSuccess)
-      return cuda_fail("moe_align: cudaFuncSetAttribute");
-    attr_set[dev] = true;
+  return launch_align(topk_ids, T, top_k, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded, capacity,
+                      stream, nullptr, nullptr, 0, nullptr, nullptr, false);
+}
+
+extern "C" int moe_route_align(const float* logits, const float* bias, int T, int E, int top_k, int block_m,
+                               int32_t* topk_ids, float* topk_weights, int32_t* sorted_token_ids,
+                               int32_t* expert_ids, int32_t* num_tokens_post_padded, int64_t capacity,
+                               moe_stream_t stream) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_route_align: need T >= 0");
+  if (E < 1 || E > kMaxExperts)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: E must be in [1, %d], got %d", kMaxExperts, E);
+  if (top_k < 1 || top_k > kRouteMaxK || top_k > E)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: top_k must be in [1, min(%d, E)], got %d", kRouteMaxK, top_k);
+  if (!valid_block_m(block_m))
+    return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: block_m must be 16, 32, 64 or 128, got %d", block_m);
+  const int64_t need = moe_align_capacity(T, top_k, E, block_m);
+  if (need >= (int64_t(1) << 31))
+    return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: T*top_k + E*(block_m-1) must be < 2^31");
+  if (capacity < need)
+    return fail(MOE_ERR_INVALID_ARG, "moe_route_align: capacity %lld < required %lld", (long long)capacity,
+                (long long)need);
+  if (capacity >= (int64_t(1) << 31))
+    return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: capacity must be < 2^31");
+  if ((T > 0 && (!logits || !topk_ids || !topk_weights)) || !sorted_token_ids || !expert_ids ||
+      !num_tokens_post_padded)
+    return fail(MOE_ERR_INVALID_ARG, "moe_route_align: null pointer");
+  const bool fused = T <= kRouteFusedMaxTokens;
+  if (!fused && T > 0) {
+    const int blocks = std::min<int64_t>((static_cast<int64_t>(T) + 7) / 8, static_cast<int64_t>(sm_count()) * 8);
+    moe_route_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(logits, bias, T, E, top_k,
+                                                                               topk_ids, topk_weights);
+    const cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return cuda_fail("moe_route_align: router launch", err);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(csize, 1, 1);
-  cfg.blockDim = dim3(kAlignThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = csize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t lerr = cudaLaunchKernelEx(&cfg, moe_align_kernel, topk_ids, R, E, block_m, sorted_token_ids,
-                                              expert_ids, num_tokens_post_padded, capacity, staged);
-  if (lerr != cudaSuccess) return cuda_fail("moe_align: launch", lerr);
-  const cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return cuda_fail("moe_align: launch", err);
-  return MOE_OK;
+  return launch_align(topk_ids, T, top_k, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded, capacity,
+                      stream, logits, bias, fused ? T : 0, topk_ids, topk_weights, !fused && T > 0);
 }

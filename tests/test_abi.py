@@ -66,6 +66,26 @@ def test_moe_align_rejects(lib):
     assert b"block_m" in lib.moe_last_error() or True
 
 
+def _route(lib, T=4, E=8, k=2, bm=64, cap=None, ptrs=(8, 8, 8, 8, 8, 8, 8), bias=None):
+    cap = lib.moe_align_capacity(T, k, E, bm) if cap is None else cap
+    return lib.moe_route_align(ptrs[0], bias, T, E, k, bm, ptrs[1], ptrs[2], ptrs[3], ptrs[4], ptrs[5], cap, None)
+
+
+def test_moe_route_align_rejects(lib):
+    assert _route(lib, k=0) == UNSUPPORTED
+    assert _route(lib, k=9) == UNSUPPORTED          # more than 8 kept experts
+    assert _route(lib, E=4, k=5) == UNSUPPORTED     # top_k > E
+    assert _route(lib, E=1025) == UNSUPPORTED
+    assert _route(lib, bm=100) == UNSUPPORTED
+    assert _route(lib, T=-1) == INVALID
+    assert _route(lib, cap=10) == INVALID
+    assert _route(lib, ptrs=(0, 8, 8, 8, 8, 8, 8)) == INVALID   # logits
+    assert _route(lib, ptrs=(8, 0, 8, 8, 8, 8, 8)) == INVALID   # topk_ids
+    assert _route(lib, ptrs=(8, 8, 0, 8, 8, 8, 8)) == INVALID   # topk_weights
+    assert _route(lib, ptrs=(8, 8, 8, 0, 8, 8, 8)) == INVALID   # sorted_token_ids
+    assert b"moe_route_align" in lib.moe_last_error()
+
+
 def test_pack_rejects(lib):
     assert lib.pack_scales_blocked(8, 8, -1, 4, 4, None) == INVALID
     assert lib.pack_scales_blocked(0, 8, 1, 4, 4, None) == INVALID

@@ -152,6 +152,18 @@ def routing(sh: Shape, seed: int = DEFAULT_SEED):
     return order.astype(np.int32), w.astype(np.float32)
 
 
+def router_logits(sh: Shape, seed: int = DEFAULT_SEED):
+    """Router inputs: (logits fp32 (T, E), per-expert bias fp32 (E,) or None).  The same draws
+    as `routing` (N(0,1) logits; on Zipf-skewed workloads bias_e = -s * ln(rank_e) over a
+    seeded rank permutation), before any routing arithmetic."""
+    logits = _rng(seed, sh, "logits").standard_normal((sh.T, sh.E), dtype=np.float32)
+    bias = None
+    if sh.zipf_s:
+        rank = _rng(seed, sh, "rank").permutation(sh.E) + 1
+        bias = (-float(sh.zipf_s) * np.log(rank.astype(np.float64))).astype(np.float32)
+    return logits, bias
+
+
 def x_f32(sh: Shape, seed: int = DEFAULT_SEED) -> np.ndarray:
     return _rng(seed, sh, "x").standard_normal((sh.T, sh.K), dtype=np.float32)
 
