@@ -77,6 +77,10 @@ def _load():
         lib.orc_fused_moe_bf16.restype = None
         lib.orc_fused_moe_mxfp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, I, P, P, I]
         lib.orc_fused_moe_mxfp8.restype = None
+        lib.orc_fused_moe_mxfp4.argtypes = lib.orc_fused_moe_mxfp8.argtypes
+        lib.orc_fused_moe_mxfp4.restype = None
+        lib.orc_e2m1_to_double.argtypes = [ctypes.c_uint8]
+        lib.orc_e2m1_to_double.restype = ctypes.c_double
         lib.orc_max_threads.argtypes = []
         lib.orc_max_threads.restype = I
         _lib = lib
@@ -230,6 +234,32 @@ def fused_moe_mxfp8(x, x_scales, w1, w1_scales, w2, w2_scales, topk_ids, topk_we
                                 _ptr(tw), T, K, N, E, top_k, None if t is None else _ptr(t), n,
                                 _ptr(out), None if f64 is None else _ptr(f64), int(nthreads))
     return (out, f64) if unrounded else out
+
+
+def fused_moe_mxfp4(x, x_scales, w1, w1_scales, w2, w2_scales, topk_ids, topk_weights,
+                    tokens=None, nthreads: int = 0, unrounded: bool = False):
+    """mxfp8 activations, MXFP4 weights: w1 (E, N, K/2) and w2 (E, K, N/4) packed e2m1 codes
+    (even index in the low nibble); scales ROW-MAJOR as for fused_moe_mxfp8."""
+    arrs = [np.ascontiguousarray(a, dtype=np.uint8) for a in (x, x_scales, w1, w1_scales, w2, w2_scales)]
+    x, xs, w1, s1, w2, s2 = arrs
+    ids = np.ascontiguousarray(topk_ids, dtype=np.int32)
+    tw = np.ascontiguousarray(topk_weights, dtype=np.float32)
+    T, K = x.shape
+    E, N, Kh = w1.shape
+    assert Kh * 2 == K and xs.shape == (T, K // 32) and s1.shape == (E, N, K // 32)
+    assert w2.shape == (E, K, N // 4) and s2.shape == (E, K, N // 64)
+    top_k = ids.shape[1]
+    t, n = _tokens_arg(tokens, T)
+    out = np.zeros((T, K), dtype=np.uint16)
+    f64 = np.zeros((T, K), dtype=np.float64) if unrounded else None
+    _load().orc_fused_moe_mxfp4(_ptr(x), _ptr(xs), _ptr(w1), _ptr(s1), _ptr(w2), _ptr(s2), _ptr(ids),
+                                _ptr(tw), T, K, N, E, top_k, None if t is None else _ptr(t), n,
+                                _ptr(out), None if f64 is None else _ptr(f64), int(nthreads))
+    return (out, f64) if unrounded else out
+
+
+def e2m1_to_double(code: int) -> float:
+    return float(_load().orc_e2m1_to_double(code))
 
 
 def max_threads() -> int:

@@ -98,6 +98,14 @@ uint8_t orc_double_to_e4m3(double x) {
   return sign | (uint8_t)(ex << 3) | (uint8_t)m;
 }
 
+/* OCP E2M1 (FP4): bias 1, one mantissa bit, no infinities or NaN; the
+ * magnitudes are 0, 0.5 (subnormal), 1, 1.5, 2, 3, 4, 6.  code is 4 bits. */
+double orc_e2m1_to_double(uint8_t code) {
+  int s = (code >> 3) & 1, ex = (code >> 1) & 3, m = code & 1;
+  double v = ex == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, ex - 1);
+  return s ? -v : v;
+}
+
 double orc_e8m0_to_double(uint8_t code) {
   if (code == 0xFF) return NAN;
   return ldexp(1.0, (int)code - 127);
@@ -365,13 +373,23 @@ void orc_fused_moe_bf16(const uint16_t* x, const uint16_t* w1, const uint16_t* w
  * fp32 (the precision the kernel holds it in), then requantised per row in
  * blocks of 32 along the intermediate dimension with the OCP MX rule, and the
  * down projection uses the dequantised requantised values.                 */
-void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
+/* Weight element idx (row-major inside one expert's matrix) decoded to its
+ * code value: e4m3 (one byte per value) or e2m1 (two values per byte, the
+ * even-indexed value in the low nibble -- reading: the usual packing order,
+ * which the pages do not state). */
+static double weight_code(const uint8_t* W, int64_t idx, int fp4) {
+  if (!fp4) return orc_e4m3_to_double(W[idx]);
+  const uint8_t b = W[idx >> 1];
+  return orc_e2m1_to_double((idx & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 0xF));
+}
+
+static void fused_moe_mx(const uint8_t* x, const uint8_t* x_scales,
                          const uint8_t* w1, const uint8_t* w1_scales,
                          const uint8_t* w2, const uint8_t* w2_scales,
                          const int32_t* topk_ids, const float* topk_weights,
                          int T, int K, int N, int E, int top_k,
                          const int32_t* tokens, int n_tokens, uint16_t* out, double* out_f64,
-                         int nthreads) {
+                         int nthreads, int fp4) {
   const int I = N / 2;
   const int KS = K / 32, IS = I / 32;
   const int count = tokens ? n_tokens : T;
@@ -395,14 +413,14 @@ void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
       for (int j = 0; j < top_k; ++j) {
         const int e = topk_ids[(int64_t)t * top_k + j];
         if (e < 0 || e >= E) continue;
-        const uint8_t* W1 = w1 + (int64_t)e * N * K;
+        const uint8_t* W1 = w1 + (int64_t)e * N * K / (fp4 ? 2 : 1);
         const uint8_t* S1 = w1_scales + (int64_t)e * N * KS;
-        const uint8_t* W2 = w2 + (int64_t)e * K * I;
+        const uint8_t* W2 = w2 + (int64_t)e * K * I / (fp4 ? 2 : 1);
         const uint8_t* S2 = w2_scales + (int64_t)e * K * IS;
         for (int n = 0; n < N; ++n) {
           double s = 0.0;
           for (int k = 0; k < K; ++k)
-            s += orc_e4m3_to_double(W1[(int64_t)n * K + k]) *
+            s += weight_code(W1, (int64_t)n * K + k, fp4) *
                  orc_e8m0_to_double(S1[(int64_t)n * KS + k / 32]) * xd[k];
           H[n] = s;
         }
@@ -413,7 +431,7 @@ void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
         for (int h = 0; h < K; ++h) {
           double s = 0.0;
           for (int i = 0; i < I; ++i)
-            s += orc_e4m3_to_double(W2[(int64_t)h * I + i]) *
+            s += weight_code(W2, (int64_t)h * I + i, fp4) *
                  orc_e8m0_to_double(S2[(int64_t)h * IS + i / 32]) * a[i];
           acc[h] += wgt * s;
         }
@@ -424,4 +442,31 @@ void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
     }
     free(xd); free(H); free(af); free(aq); free(as); free(a); free(acc);
   }
+}
+
+void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
+                         const uint8_t* w1, const uint8_t* w1_scales,
+                         const uint8_t* w2, const uint8_t* w2_scales,
+                         const int32_t* topk_ids, const float* topk_weights,
+                         int T, int K, int N, int E, int top_k,
+                         const int32_t* tokens, int n_tokens, uint16_t* out, double* out_f64,
+                         int nthreads) {
+  fused_moe_mx(x, x_scales, w1, w1_scales, w2, w2_scales, topk_ids, topk_weights, T, K, N, E, top_k, tokens,
+               n_tokens, out, out_f64, nthreads, 0);
+}
+
+/* MXFP4 weights (e2m1 values, e8m0 scale per 32 along the contraction
+ * dimension) with mxfp8 activations: the same forward as the mxfp8 path,
+ * the weights decoded from packed e2m1 codes.  DeepGEMM #411 "SM90 FP8 x
+ * MXFP4 MegaMoE" runs this activation/weight pairing; the OCP MX v1.0 FP4
+ * element format defines the codes. */
+void orc_fused_moe_mxfp4(const uint8_t* x, const uint8_t* x_scales,
+                         const uint8_t* w1, const uint8_t* w1_scales,
+                         const uint8_t* w2, const uint8_t* w2_scales,
+                         const int32_t* topk_ids, const float* topk_weights,
+                         int T, int K, int N, int E, int top_k,
+                         const int32_t* tokens, int n_tokens, uint16_t* out, double* out_f64,
+                         int nthreads) {
+  fused_moe_mx(x, x_scales, w1, w1_scales, w2, w2_scales, topk_ids, topk_weights, T, K, N, E, top_k, tokens,
+               n_tokens, out, out_f64, nthreads, 1);
 }

@@ -27,6 +27,7 @@ double orc_bf16_to_double(uint16_t bits);
 uint16_t orc_double_to_bf16(double x);          /* round to nearest even */
 double orc_e4m3_to_double(uint8_t code);        /* OCP E4M3 (fn): NaN for 0x7F/0xFF */
 uint8_t orc_double_to_e4m3(double x);           /* RNE, saturate to +-448 */
+double orc_e2m1_to_double(uint8_t code);        /* OCP E2M1 (FP4), 4-bit code */
 double orc_e8m0_to_double(uint8_t code);        /* 2^(code-127); NaN for 0xFF */
 /* OCP MX block scale for a block whose largest magnitude is amax (fp32). */
 uint8_t orc_mx_scale_byte(float amax);
@@ -63,6 +64,17 @@ void orc_fused_moe_bf16(const uint16_t* x, const uint16_t* w1, const uint16_t* w
 
 /* w1_scales / w2_scales are ROW-MAJOR here: (E, N, K/32) and (E, K, (N/2)/32). */
 void orc_fused_moe_mxfp8(const uint8_t* x, const uint8_t* x_scales,
+                         const uint8_t* w1, const uint8_t* w1_scales,
+                         const uint8_t* w2, const uint8_t* w2_scales,
+                         const int32_t* topk_ids, const float* topk_weights,
+                         int T, int K, int N, int E, int top_k,
+                         const int32_t* tokens, int n_tokens, uint16_t* out, double* out_f64,
+                         int nthreads);
+
+/* As orc_fused_moe_mxfp8 with MXFP4 weights: w1 (E, N, K/2) and w2
+ * (E, K, N/4) bytes of packed e2m1 codes (even index in the low nibble),
+ * scales as for mxfp8. */
+void orc_fused_moe_mxfp4(const uint8_t* x, const uint8_t* x_scales,
                          const uint8_t* w1, const uint8_t* w1_scales,
                          const uint8_t* w2, const uint8_t* w2_scales,
                          const int32_t* topk_ids, const float* topk_weights,

@@ -15,7 +15,14 @@ C2     bf16     4096  4096  256   6      128      64, 256
 C3     mxfp8    4096  4096  288   8      128      64 ... 8192
 C4     mxfp8    7168  6144  384   6      128      1024 ... 8192
 C5     bf16     4096  512   128   8      128      1, 8, 64, 512, 8192 (Zipf bias)
+C3F4   mxfp4    4096  4096  288   8      128      64 ... 8192 (C3 with MXFP4 weights)
+C4F4   mxfp4    7168  6144  384   6      128      1024 ... 8192 (C4 with MXFP4 weights)
 =====  =======  ====  ====  ====  =====  =======  ===========================
+
+The two F4 workloads draw the same fp32 tensors as C3 / C4 and quantise the
+weights to MXFP4 (e2m1 values, e8m0 scale per 32 along K, two values per byte,
+the even-indexed value in the low nibble) instead of mxfp8; activations stay
+mxfp8.
 
 Recipe (all fp32 draws from numpy PCG64 streams keyed by
 ``SeedSequence([seed, workload, tensor, expert])``):
@@ -51,7 +58,13 @@ _WORKLOADS = {
                Ts=(1024, 2048, 4096, 8192), zipf_s=None),
     "C5": dict(dtype="bf16", K=4096, N=512, E=128, top_k=8, block_m=128,
                Ts=(1, 8, 64, 512, 8192), zipf_s=1.2),
+    "C3F4": dict(dtype="mxfp4", K=4096, N=4096, E=288, top_k=8, block_m=128,
+                 Ts=(64, 256, 1024, 2048, 4096, 8192), zipf_s=None),
+    "C4F4": dict(dtype="mxfp4", K=7168, N=6144, E=384, top_k=6, block_m=128,
+                 Ts=(1024, 2048, 4096, 8192), zipf_s=None),
 }
+# random streams: the F4 workloads share their base workload's draws
+_STREAM_KEY = {"C1": 1, "C2": 2, "C3": 3, "C4": 4, "C5": 5, "C3F4": 3, "C4F4": 4}
 _TENSOR_IDS = {"x": 1, "w1": 2, "w2": 3, "logits": 4, "rank": 5}
 
 
@@ -93,7 +106,7 @@ def shape(name: str, T: int | None = None, **override) -> Shape:
 
 
 def _rng(seed: int, sh: Shape, tensor: str, expert: int = 0) -> np.random.Generator:
-    key = [int(seed), int(sh.name[1:]) if sh.name[1:].isdigit() else 0, _TENSOR_IDS[tensor],
+    key = [int(seed), _STREAM_KEY.get(sh.name, 0), _TENSOR_IDS[tensor],
            int(expert), int(sh.T) if tensor in ("x", "logits") else 0]
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence(key)))
 
@@ -216,11 +229,60 @@ def bf16_inputs(sh: Shape, seed: int = DEFAULT_SEED, threads: int | None = None)
                 w2=bf16_weights(sh, "w2", seed, threads), topk_ids=ids, topk_weights=tw)
 
 
+# OCP E2M1 magnitudes by 3-bit code (exponent bias 1, one mantissa bit)
+_E2M1_MAG = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
+
+
+def mx_quantize_fp4(v: np.ndarray):
+    """Caller-side OCP MX FP4 quantiser: (..., L) fp32 -> packed e2m1 codes (..., L/2) u8 (value
+    2j in the low nibble of byte j) and e8m0 scales (..., L/32).  Shared scale
+    2^(floor(log2 amax) - 2) (emax of e2m1 is 2); values rounded to the nearest e2m1 magnitude,
+    ties to the even code, beyond 6 saturated; an all-zero block gets scale byte 0."""
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    L = v.shape[-1]
+    assert L % 32 == 0
+    blk = v.reshape(-1, 32).astype(np.float64)
+    amax = np.abs(blk).max(axis=1)
+    _, ex = np.frexp(amax)
+    shared = np.where(amax > 0, ex.astype(np.int32) - 1 - 2, -127)
+    shared = np.clip(shared, -127, 127)
+    scaled = blk * np.ldexp(1.0, -shared)[:, None]
+    mag = np.abs(scaled)
+    # nearest magnitude by exhaustive comparison; on a tie the even code (smaller index with
+    # an even mantissa bit) wins
+    d = np.abs(mag[..., None] - _E2M1_MAG[None, None, :])
+    best = np.argmin(d, axis=-1)
+    dmin = np.take_along_axis(d, best[..., None], axis=-1)[..., 0]
+    nxt = np.minimum(best + 1, 7)
+    tie = (np.take_along_axis(d, nxt[..., None], axis=-1)[..., 0] == dmin) & (nxt != best)
+    best = np.where(tie & (best % 2 == 1), nxt, best)
+    best = np.where(mag >= 6.0, 7, best)
+    codes = (best | np.where(np.signbit(scaled), 8, 0)).astype(np.uint8).reshape(v.shape)
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    scales = (shared + 127).astype(np.uint8).reshape(v.shape[:-1] + (L // 32,))
+    return packed, scales
+
+
+def mxfp4_weights(sh: Shape, which: str, seed: int = DEFAULT_SEED, threads: int | None = None):
+    """(packed e2m1 (E, rows, cols/2) u8, row-major scales (E, rows, cols/32) u8)."""
+    rows, cols = (sh.N, sh.K) if which == "w1" else (sh.K, sh.I)
+    codes = np.empty((sh.E, rows, cols // 2), dtype=np.uint8)
+    scales = np.empty((sh.E, rows, cols // 32), dtype=np.uint8)
+
+    def put(e, v, o):
+        c, s = mx_quantize_fp4(v)
+        o[0][e] = c
+        o[1][e] = s
+    _fill_experts(sh, which, put, (codes, scales), seed, threads)
+    return codes, scales
+
+
 def mxfp8_inputs(sh: Shape, seed: int = DEFAULT_SEED, threads: int | None = None) -> dict:
     ids, tw = routing(sh, seed)
     xq, xs = mx_quantize_inputs(x_f32(sh, seed))
-    w1, s1 = mxfp8_weights(sh, "w1", seed, threads)
-    w2, s2 = mxfp8_weights(sh, "w2", seed, threads)
+    wq = mxfp4_weights if sh.dtype == "mxfp4" else mxfp8_weights
+    w1, s1 = wq(sh, "w1", seed, threads)
+    w2, s2 = wq(sh, "w2", seed, threads)
     return dict(x=xq, x_scales=xs, w1=w1, w1_scales=s1, w2=w2, w2_scales=s2, topk_ids=ids, topk_weights=tw)
 
 
