@@ -86,7 +86,8 @@ def cost_model(sh: W.Shape, topk_ids: np.ndarray, peaks: dict):
     counts = np.bincount(topk_ids.reshape(-1)[(topk_ids.reshape(-1) >= 0) & (topk_ids.reshape(-1) < sh.E)],
                          minlength=sh.E)
     touched = int((counts > 0).sum())
-    b = 2.0 if sh.dtype == "bf16" else 1.0 + 1.0 / 32.0
+    # weight bytes per value: bf16 2; mxfp8 1 + 1/32 (e8m0 per 32); MXFP4 1/2 + 1/32
+    b = {"bf16": 2.0, "mxfp8": 1.0 + 1.0 / 32.0, "mxfp4": 0.5 + 1.0 / 32.0}[sh.dtype]
     bytes_w = touched * 1.5 * sh.N * sh.K * b
     p_tc = peaks["bf16_tflops"] * (1.0 if sh.dtype == "bf16" else 2.0) * 1e12
     bw = peaks["hbm_gbs"] * 1e9
@@ -205,8 +206,9 @@ def _run_oracle(sh, inp, toks, thr):
     if sh.dtype == "bf16":
         return oracle.fused_moe_bf16(inp["x"], inp["w1"], inp["w2"], inp["topk_ids"], inp["topk_weights"],
                                      tokens=toks, nthreads=thr)
-    return oracle.fused_moe_mxfp8(inp["x"], inp["x_scales"], inp["w1"], inp["w1_scales"], inp["w2"],
-                                  inp["w2_scales"], inp["topk_ids"], inp["topk_weights"], tokens=toks, nthreads=thr)
+    fwd = oracle.fused_moe_mxfp4 if sh.dtype == "mxfp4" else oracle.fused_moe_mxfp8
+    return fwd(inp["x"], inp["x_scales"], inp["w1"], inp["w1_scales"], inp["w2"], inp["w2_scales"],
+               inp["topk_ids"], inp["topk_weights"], tokens=toks, nthreads=thr)
 
 
 def run_reference(args):
@@ -285,7 +287,7 @@ class Problem:
             self.x, self.xs, self.w1, self.w2 = up(inp["x"]), up(inp["x_scales"]), up(inp["w1"]), up(inp["w2"])
             self.s1 = moe.pack_scales_blocked(up(inp["w1_scales"]))
             self.s2 = moe.pack_scales_blocked(up(inp["w2_scales"]))
-            dt = moe.DTYPE_MXFP8
+            dt = moe.DTYPE_MXFP4 if sh.dtype == "mxfp4" else moe.DTYPE_MXFP8
         self.ws = torch.empty(moe.moe_workspace_bytes(dt, sh.T, sh.K, sh.N, sh.E, sh.top_k, bm),
                               dtype=torch.uint8, device=dev)
         self.plain = moe.Tuning(stages, ctas, None)
@@ -300,8 +302,9 @@ class Problem:
             m.fused_moe_bf16(self.x, self.w1, self.w2, self.s_ids, self.e_ids, self.ntpp, self.tw, self.out, self.bm,
                              workspace=self.ws, tune=tune)
         else:
-            m.fused_moe_mxfp8(self.x, self.xs, self.w1, self.s1, self.w2, self.s2, self.s_ids, self.e_ids, self.ntpp,
-                              self.tw, self.out, self.bm, workspace=self.ws, tune=tune)
+            fwd = m.fused_moe_mxfp4 if self.sh.dtype == "mxfp4" else m.fused_moe_mxfp8
+            fwd(self.x, self.xs, self.w1, self.s1, self.w2, self.s2, self.s_ids, self.e_ids, self.ntpp,
+                self.tw, self.out, self.bm, workspace=self.ws, tune=tune)
 
     def step(self, tune=None, plan_event=None):
         if plan_event is not None:
@@ -408,7 +411,7 @@ def measure_e2e(prob: Problem, steps: int, barrier=None):
         host_in = [hx.pin_memory(), torch.from_numpy(inp["topk_ids"]).pin_memory(),
                    torch.from_numpy(inp["topk_weights"]).pin_memory()]
         dev_in = [prob.x, prob.ids, prob.tw]
-    if sh.dtype == "mxfp8":
+    if sh.dtype != "bf16":
         host_in.append(torch.from_numpy(np.ascontiguousarray(inp["x_scales"])).pin_memory())
         dev_in.append(prob.xs)
     host_out = torch.empty((sh.T, sh.K), dtype=torch.bfloat16).pin_memory()

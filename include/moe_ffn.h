@@ -59,7 +59,7 @@ enum {
   MOE_ERR_TIMEOUT = -6      /* a device-side bounded wait ran out          */
 };
 
-enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_MXFP8 = 1 };
+enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_MXFP8 = 1, MOE_DTYPE_MXFP4 = 2 };
 
 /* Message describing the last error returned on the calling host thread. */
 MOE_API const char* moe_last_error(void);
@@ -202,6 +202,29 @@ MOE_API int fused_moe_bf16(const void* x, const void* w1, const void* w2,
  * ---------------------------------------------------------------------- */
 MOE_API int fused_moe_mxfp8(const uint8_t* x_e4m3, const uint8_t* x_scales, const uint8_t* w1_e4m3,
                     const uint8_t* w1_scales_blocked, const uint8_t* w2_e4m3,
+                    const uint8_t* w2_scales_blocked, const int32_t* sorted_token_ids,
+                    const int32_t* expert_ids, const int32_t* num_tokens_post_padded,
+                    const float* topk_weights, void* out, int T, int K, int N, int E, int top_k,
+                    int block_m, int64_t capacity, void* workspace, int64_t workspace_bytes,
+                    const moe_tuning* tune, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * fused_moe_mxfp4 -- mxfp8 activations with MXFP4 weights (DeepGEMM #411
+ * "SM90 FP8 x MXFP4 MegaMoE" pairs these operand formats; the element format
+ * is OCP MX v1.0 FP4, E2M1).  The forward is fused_moe_mxfp8's; only the
+ * weight encoding differs: e2m1 values (sign, 2 exponent bits with bias 1,
+ * 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) with one e8m0
+ * scale per 32 along the contraction dimension, two values per byte, the
+ * even-indexed value in the low nibble.  Half the weight bytes of mxfp8.
+ *
+ *   w1_e2m1 (E, N, K/2) u8      w1_scales_blocked as for fused_moe_mxfp8
+ *   w2_e2m1 (E, K, N/4) u8      w2_scales_blocked as for fused_moe_mxfp8
+ *   other arguments as fused_moe_mxfp8; workspace from
+ *   moe_workspace_bytes(MOE_DTYPE_MXFP4, ...).
+ * Constraints: as fused_moe_mxfp8, plus w1 and w2 32-byte aligned.
+ * ---------------------------------------------------------------------- */
+MOE_API int fused_moe_mxfp4(const uint8_t* x_e4m3, const uint8_t* x_scales, const uint8_t* w1_e2m1,
+                    const uint8_t* w1_scales_blocked, const uint8_t* w2_e2m1,
                     const uint8_t* w2_scales_blocked, const int32_t* sorted_token_ids,
                     const int32_t* expert_ids, const int32_t* num_tokens_post_padded,
                     const float* topk_weights, void* out, int T, int K, int N, int E, int top_k,

@@ -18,6 +18,8 @@ Entry points (same names as the C ABI):
 * ``fused_moe_bf16`` / ``fused_moe_mxfp8`` -- gather, gate/up GEMM, SwiGLU
   (mxfp8: on-chip requant of the intermediate), down GEMM and the top-k
   weighted reduction into ``out`` ("Prime Flash MoE", intro / API / Shapes).
+* ``fused_moe_mxfp4`` -- the mxfp8 forward with MXFP4 (e2m1) weights, two
+  values per byte (DeepGEMM #411 "SM90 FP8 x MXFP4 MegaMoE" operand pairing).
 * ``pack_scales_blocked`` -- weight scales into 512-byte tiles of
   128 MN x 128 K ("Prime Flash MoE", Scale layout (mxfp8)).
 """
@@ -31,6 +33,7 @@ from . import _build
 
 __all__ = [
     "MoeError", "load", "moe_align", "moe_align_capacity", "moe_route_align", "fused_moe_bf16", "fused_moe_mxfp8",
+    "fused_moe_mxfp4", "DTYPE_MXFP4",
     "pack_scales_blocked", "pack_scales_blocked_bytes", "moe_workspace_bytes", "moe_device_status",
     "Tuning", "DTYPE_BF16", "DTYPE_MXFP8", "LIB_PATH", "fused_moe_bf16_noalloc",
     "fused_moe_bf16_noalloc_max_workspace",
@@ -38,6 +41,7 @@ __all__ = [
 
 DTYPE_BF16 = 0
 DTYPE_MXFP8 = 1
+DTYPE_MXFP4 = 2
 LIB_PATH = _build.LIB
 
 _ERRORS = {-1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_ALIGNMENT",
@@ -87,6 +91,8 @@ _SIGS = {
     "moe_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I], _I64),
     "fused_moe_bf16": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _I64, _P, _P], _I),
     "fused_moe_mxfp8": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _I64,
+                         _P, _P], _I),
+    "fused_moe_mxfp4": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _I64,
                          _P, _P], _I),
     "fused_moe_bf16_noalloc_max_workspace": ([], _I64),
     "fused_moe_bf16_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _P], _I),
@@ -302,6 +308,36 @@ def fused_moe_mxfp8(x, x_scales, w1, w1_scales_blocked, w2, w2_scales_blocked, s
     top_k = topk_weights.shape[1]
     ws = _workspace(DTYPE_MXFP8, T, K, N, E, top_k, block_m, workspace, x.device)
     _check(load().fused_moe_mxfp8(
+        _ptr(x), _ptr(x_scales), _ptr(w1), _ptr(w1_scales_blocked), _ptr(w2), _ptr(w2_scales_blocked),
+        _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(topk_weights), _ptr(out),
+        T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws), ws.numel(),
+        None if tune is None else ctypes.byref(tune), _stream(stream)))
+    return out
+
+
+def fused_moe_mxfp4(x, x_scales, w1, w1_scales_blocked, w2, w2_scales_blocked, sorted_token_ids, expert_ids,
+                    num_tokens_post_padded, topk_weights, out, block_m: int, workspace=None,
+                    tune: Tuning | None = None, stream=None):
+    """mxfp8 activations, MXFP4 weights: w1 (E, N, K/2) and w2 (E, K, N/4) uint8 of packed e2m1 codes
+    (even index in the low nibble); scales and the rest as fused_moe_mxfp8."""
+    import torch
+
+    _need(x, "x", (torch.uint8, torch.float8_e4m3fn))
+    for t, n in ((w1, "w1"), (w2, "w2"), (x_scales, "x_scales"), (w1_scales_blocked, "w1_scales_blocked"),
+                 (w2_scales_blocked, "w2_scales_blocked")):
+        _need(t, n, (torch.uint8,))
+    _need(out, "out", (torch.bfloat16,))
+    _need(topk_weights, "topk_weights", (torch.float32,))
+    for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
+                 (num_tokens_post_padded, "num_tokens_post_padded")):
+        _need(t, n, (torch.int32,))
+    T, K = x.shape
+    E, N, Kh = w1.shape
+    if Kh * 2 != K:
+        raise ValueError("w1 must be (E, N, K/2) packed e2m1")
+    top_k = topk_weights.shape[1]
+    ws = _workspace(DTYPE_MXFP4, T, K, N, E, top_k, block_m, workspace, x.device)
+    _check(load().fused_moe_mxfp4(
         _ptr(x), _ptr(x_scales), _ptr(w1), _ptr(w1_scales_blocked), _ptr(w2), _ptr(w2_scales_blocked),
         _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(topk_weights), _ptr(out),
         T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws), ws.numel(),

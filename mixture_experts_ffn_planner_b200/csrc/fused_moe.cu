@@ -101,6 +101,7 @@ struct P1Params {
   int max_blocks;           // blocks a kernel may visit
   int w_reuse;              // 1: experts average more than one planner block (weights re-read)
   float* part;              // split-K partials: [kMaxSplitItems][kSplitRows][256] fp32
+  int w_fp4;                // weights are MXFP4: e2m1 codes, half the bytes per copy
   int n_jt;                 // ceil(I / 128): work units per planner block
   int stages, stage_bytes;
   int off_b, off_sf;        // stage offsets of the B tile and of the scale tiles
@@ -122,6 +123,7 @@ struct P2Params {
   int n_ht;                 // ceil(K / 256): work units per planner block
   int n_kc;                 // K-chunks of the down GEMM
   int a_full;               // the stage's A region holds 128 rows
+  int w_fp4;                // weights are MXFP4 (as in the gate/up phase)
   int stages, stage_bytes;
   int off_b, off_sf;
 };
@@ -324,7 +326,10 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     // together, so the tiles keep normal L2 priority; otherwise each is read
     // once and is evicted first.
     const uint64_t pol = p.w_reuse ? policy_evict_normal() : policy_evict_first();
-    const uint32_t tx = 2 * kTI * kRowBytes + (kFp8 ? 2 * kSfTileBytes : 0);
+    // an MXFP4 weight row of a stage is 64 packed bytes, expanded by the copy
+    // into the 128-byte row of the unpacked form the MMA reads
+    const uint32_t w_row_bytes = p.w_fp4 ? kRowBytes / 2 : kRowBytes;
+    const uint32_t tx = 2 * kTI * w_row_bytes + (kFp8 ? 2 * kSfTileBytes : 0);
     const int MT1 = p.N / 128, KT1 = p.K / 128;
     int s = 0;
     uint32_t ph = 0;
@@ -409,8 +414,8 @@ __global__ void __launch_bounds__(kP1Threads, 1)
               const uint64_t step = static_cast<uint64_t>(2 * kk);  // 32 bytes along K
               if (kFp8) {
                 const uint32_t sfid = static_cast<uint32_t>(kk) << 30;
-                mma_mxf8(d, ad + step, bd + step, idesc_mxf8(kM, 256, kk, kk), (tbase + kSfaCol) | sfid,
-                         (tbase + kSfbCol) | sfid, acc);
+                mma_mxf8(d, ad + step, bd + step, idesc_mxf8(kM, 256, kk, kk, p.w_fp4 ? kFmtE2M1 : kFmtE4M3),
+                         (tbase + kSfaCol) | sfid, (tbase + kSfbCol) | sfid, acc);
               } else {
                 mma_f16(d, ad + step, bd + step, kIdesc, acc);
               }
@@ -766,7 +771,8 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       // per stage than 16-row and 128-row pieces.
       const bool big_a = p.a_full && bi.n16 >= 64;
       const int a_rows = big_a ? 128 : bi.n16;
-      const uint32_t tx = nb * 128 * kRowBytes + a_rows * kRowBytes + (kFp8 ? (1 + nb) * kSfTileBytes : 0);
+      const uint32_t w_row_bytes = p.w_fp4 ? kRowBytes / 2 : kRowBytes;  // packed MXFP4 rows
+      const uint32_t tx = nb * 128 * w_row_bytes + a_rows * kRowBytes + (kFp8 ? (1 + nb) * kSfTileBytes : 0);
       for (int kc = 0; kc < p.n_kc; ++kc) {
         if (lane == 0) {
           ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
@@ -838,8 +844,8 @@ __global__ void __launch_bounds__(kP2Threads, 1)
               const uint64_t step = static_cast<uint64_t>(2 * kk);
               if (kFp8) {
                 const uint32_t sfid = static_cast<uint32_t>(kk) << 30;
-                mma_mxf8(d, ad + step, bd + step, idesc_mxf8(kM, nn, kk, kk), (tbase + kSfaCol) | sfid,
-                         (tbase + kSfbCol) | sfid, acc);
+                mma_mxf8(d, ad + step, bd + step, idesc_mxf8(kM, nn, kk, kk, p.w_fp4 ? kFmtE2M1 : kFmtE4M3),
+                         (tbase + kSfaCol) | sfid, (tbase + kSfbCol) | sfid, acc);
               } else {
                 mma_f16(d, ad + step, bd + step, idesc_bf16(kM, nn), acc);
               }
@@ -1138,15 +1144,25 @@ static EncodeTiledFn get_encode() {
 }
 
 // 2-D row-major [rows x cols] tensor, box [box_rows x 128 bytes], 128-byte swizzle.
-static int make_tmap(CUtensorMap* m, const void* base, bool fp8, int64_t rows, int64_t cols, int box_rows) {
+// Element kinds of the 2-D tensor maps: bf16, one-byte codes (e4m3 / e8m0),
+// and packed e2m1 pairs, which the copy expands into the unpacked form (each
+// 16 values' 8 bytes followed by an 8-byte gap) that the block-scaled MMA
+// reads as one byte per value; a box row is then 128 values in both cases.
+enum TmapKind { kTmBf16, kTmU8, kTmFp4 };
+
+static int make_tmap(CUtensorMap* m, const void* base, TmapKind kind, int64_t rows, int64_t cols, int box_rows) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
-  const int esize = fp8 ? 1 : 2;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * esize)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(kRowBytes / esize), static_cast<cuuint32_t>(box_rows)};
+  const int64_t row_bytes = kind == kTmBf16 ? cols * 2 : (kind == kTmU8 ? cols : cols / 2);
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kind == kTmBf16 ? kRowBytes / 2 : kRowBytes),
+                       static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  const CUtensorMapDataType dt = kind == kTmBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : kind == kTmU8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                 : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
+  const CUresult r = enc(m, dt, 2,
                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1170,6 +1186,7 @@ static int set_smem_attr(K kernel, int bytes, bool* done) {
 
 struct FusedArgs {
   bool fp8;
+  bool w_fp4;  // mxfp8 activations with MXFP4 weights
   const void* x;
   const uint8_t* x_sf;
   const void* w1;
@@ -1208,7 +1225,7 @@ static int pick_stages(int stage_bytes, int ctrl, int requested, int max_stages)
 }
 
 static int run_fused(const FusedArgs& a) {
-  const char* nm = a.fp8 ? "fused_moe_mxfp8" : "fused_moe_bf16";
+  const char* nm = a.w_fp4 ? "fused_moe_mxfp4" : (a.fp8 ? "fused_moe_mxfp8" : "fused_moe_bf16");
   if (a.T < 0 || a.K <= 0 || a.N <= 0 || a.E < 1 || a.top_k < 1)
     return fail(MOE_ERR_INVALID_ARG, "%s: need T >= 0, K > 0, N > 0, E >= 1, top_k >= 1", nm);
   if (!valid_block_m(a.bm)) return fail(MOE_ERR_UNSUPPORTED, "%s: block_m must be 16, 32, 64 or 128", nm);
@@ -1234,6 +1251,8 @@ static int run_fused(const FusedArgs& a) {
       !aligned(a.ws, 256) || (a.fp8 && (!aligned(a.x_sf, 16) || !aligned(a.w1_sf, 16) || !aligned(a.w2_sf, 16))) ||
       !aligned(a.sorted_ids, 4) || !aligned(a.expert_ids, 4) || !aligned(a.ntpp, 4) || !aligned(a.topk_w, 4))
     return fail(MOE_ERR_ALIGNMENT, "%s: tensors must be 16-byte aligned and the workspace 256-byte aligned", nm);
+  if (a.w_fp4 && (!aligned(a.w1, 32) || !aligned(a.w2, 32)))
+    return fail(MOE_ERR_ALIGNMENT, "%s: packed e2m1 weights must be 32-byte aligned", nm);
   const WsLayout L = ws_layout(a.fp8, a.T, a.K, a.N, a.E, a.top_k, a.bm);
   if (a.ws_bytes < L.total)
     return fail(MOE_ERR_WORKSPACE, "%s: workspace %lld bytes < required %lld", nm, (long long)a.ws_bytes,
@@ -1253,17 +1272,18 @@ static int run_fused(const FusedArgs& a) {
 
   CUtensorMap tm_w1, tm_w2, tm_w2x, tm_act, tm_actx;
   int rc;
-  if ((rc = make_tmap(&tm_w1, a.w1, a.fp8, static_cast<int64_t>(a.E) * a.N, a.K, 128)) != MOE_OK) return rc;
-  if ((rc = make_tmap(&tm_w2, a.w2, a.fp8, static_cast<int64_t>(a.E) * a.K, I, 128)) != MOE_OK) return rc;
-  if ((rc = make_tmap(&tm_act, ws + L.act, a.fp8, L.cap_rows, I, 16)) != MOE_OK) return rc;
+  const TmapKind wk = a.w_fp4 ? kTmFp4 : (a.fp8 ? kTmU8 : kTmBf16), ak = a.fp8 ? kTmU8 : kTmBf16;
+  if ((rc = make_tmap(&tm_w1, a.w1, wk, static_cast<int64_t>(a.E) * a.N, a.K, 128)) != MOE_OK) return rc;
+  if ((rc = make_tmap(&tm_w2, a.w2, wk, static_cast<int64_t>(a.E) * a.K, I, 128)) != MOE_OK) return rc;
+  if ((rc = make_tmap(&tm_act, ws + L.act, ak, L.cap_rows, I, 16)) != MOE_OK) return rc;
   // the one-box forms are encoded only where the down phase can use them
   // (full 256-feature tiles; 128-row A regions)
   tm_w2x = tm_w2;
   tm_actx = tm_act;
   const int a_rows = a_region_rows(a.bm, static_cast<int64_t>(a.T) * a.top_k);
-  if (a.K >= 2 * 128 && (rc = make_tmap(&tm_w2x, a.w2, a.fp8, static_cast<int64_t>(a.E) * a.K, I, 256)) != MOE_OK)
+  if (a.K >= 2 * 128 && (rc = make_tmap(&tm_w2x, a.w2, wk, static_cast<int64_t>(a.E) * a.K, I, 256)) != MOE_OK)
     return rc;
-  if (a_rows >= kM && (rc = make_tmap(&tm_actx, ws + L.act, a.fp8, L.cap_rows, I, 128)) != MOE_OK) return rc;
+  if (a_rows >= kM && (rc = make_tmap(&tm_actx, ws + L.act, ak, L.cap_rows, I, 128)) != MOE_OK) return rc;
 
   const int nsm = sm_count();
   if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(SM count)");
@@ -1289,6 +1309,7 @@ static int run_fused(const FusedArgs& a) {
   p1.R = a.T * a.top_k;
   p1.max_blocks = max_blocks;
   p1.w_reuse = static_cast<int64_t>(a.T) * a.top_k >= static_cast<int64_t>(a.E) * a.bm ? 1 : 0;
+  p1.w_fp4 = a.w_fp4 ? 1 : 0;
   p1.n_jt = (I + kTI - 1) / kTI;
   p1.stage_bytes = stage_bytes(a.fp8, a_rows);
   p1.off_b = off_b_of(a_rows);
@@ -1308,6 +1329,7 @@ static int run_fused(const FusedArgs& a) {
   p2.K = a.K; p2.I = I; p2.E = a.E; p2.top_k = a.top_k; p2.bm = a.bm; p2.R = p1.R;
   p2.max_blocks = max_blocks;
   p2.w_reuse = p1.w_reuse;
+  p2.w_fp4 = p1.w_fp4;
   p2.n_ht = (a.K + kTH - 1) / kTH;
   p2.n_kc = a.fp8 ? I / 128 : (I + 63) / 64;
   p2.stage_bytes = stage_bytes(a.fp8, a_rows);
@@ -1406,8 +1428,8 @@ using namespace moe;
 
 extern "C" int64_t moe_workspace_bytes(int dtype, int T, int K, int N, int E, int top_k, int block_m) {
   if (T < 0 || K <= 0 || N <= 0 || E < 1 || top_k < 1 || !valid_block_m(block_m)) return -1;
-  if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_MXFP8) return -1;
-  return ws_layout(dtype == MOE_DTYPE_MXFP8, T, K, N, E, top_k, block_m).total;
+  if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_MXFP8 && dtype != MOE_DTYPE_MXFP4) return -1;
+  return ws_layout(dtype != MOE_DTYPE_BF16, T, K, N, E, top_k, block_m).total;
 }
 
 extern "C" int moe_device_status(moe_stream_t stream) {
@@ -1452,6 +1474,26 @@ extern "C" int fused_moe_mxfp8(const uint8_t* x_e4m3, const uint8_t* x_scales, c
   a.fp8 = true;
   a.x = x_e4m3; a.x_sf = x_scales; a.w1 = w1_e4m3; a.w1_sf = w1_scales_blocked;
   a.w2 = w2_e4m3; a.w2_sf = w2_scales_blocked;
+  a.sorted_ids = sorted_token_ids; a.expert_ids = expert_ids; a.ntpp = num_tokens_post_padded;
+  a.topk_w = topk_weights; a.out = out;
+  a.T = T; a.K = K; a.N = N; a.E = E; a.top_k = top_k; a.bm = block_m; a.capacity = capacity;
+  a.ws = workspace; a.ws_bytes = workspace_bytes; a.tune = tune;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  return run_fused(a);
+}
+
+extern "C" int fused_moe_mxfp4(const uint8_t* x_e4m3, const uint8_t* x_scales, const uint8_t* w1_e2m1,
+                               const uint8_t* w1_scales_blocked, const uint8_t* w2_e2m1,
+                               const uint8_t* w2_scales_blocked, const int32_t* sorted_token_ids,
+                               const int32_t* expert_ids, const int32_t* num_tokens_post_padded,
+                               const float* topk_weights, void* out, int T, int K, int N, int E, int top_k,
+                               int block_m, int64_t capacity, void* workspace, int64_t workspace_bytes,
+                               const moe_tuning* tune, moe_stream_t stream) {
+  FusedArgs a{};
+  a.fp8 = true;
+  a.w_fp4 = true;
+  a.x = x_e4m3; a.x_sf = x_scales; a.w1 = w1_e2m1; a.w1_sf = w1_scales_blocked;
+  a.w2 = w2_e2m1; a.w2_sf = w2_scales_blocked;
   a.sorted_ids = sorted_token_ids; a.expert_ids = expert_ids; a.ntpp = num_tokens_post_padded;
   a.topk_w = topk_weights; a.out = out;
   a.T = T; a.K = K; a.N = N; a.E = E; a.top_k = top_k; a.bm = block_m; a.capacity = capacity;

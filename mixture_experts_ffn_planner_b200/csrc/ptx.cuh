@@ -269,10 +269,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Instruction descriptor, kind::mxf8f6f4 block-scaled: A and B e4m3,
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: A e4m3, B e4m3
+// (b_fmt 0) or e2m1 (b_fmt 5, read from the unpacked shared-memory form),
 // K-major, e8m0 scales; sf ids pick the byte of the 32-bit TMEM scale word.
-__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sfa_id, uint32_t sfb_id) {
-  return (sfb_id << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sfa_id, uint32_t sfb_id,
+                                                  uint32_t b_fmt = kFmtE4M3) {
+  return (sfb_id << 4) | (kFmtE4M3 << 7) | (b_fmt << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
          (static_cast<uint32_t>(M >> 4) << 24) | (sfa_id << 29);
 }
 

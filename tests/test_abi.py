@@ -103,6 +103,22 @@ def _mx(lib, T=64, K=1024, N=1024, E=8, k=2, bm=128, p=256, ws=1 << 30):
     return lib.fused_moe_mxfp8(p, p, p, p, p, p, p, p, p, p, p, T, K, N, E, k, bm, cap, p, ws, None, None)
 
 
+def _mx4(lib, T=64, K=1024, N=1024, E=8, k=2, bm=128, p=256, w=256, ws=1 << 30):
+    cap = lib.moe_align_capacity(T, k, E, bm)
+    return lib.fused_moe_mxfp4(p, p, w, p, w, p, p, p, p, p, p, T, K, N, E, k, bm, cap, p, ws, None, None)
+
+
+def test_mxfp4_rejects(lib):
+    assert _mx4(lib, K=1152) == UNSUPPORTED
+    assert _mx4(lib, N=640) == UNSUPPORTED
+    assert _mx4(lib, p=0) == INVALID
+    assert _mx4(lib, w=256 + 16) == ALIGNMENT      # packed e2m1 weights need 32-byte alignment
+    assert _mx4(lib, ws=4096) == WORKSPACE
+    assert b"fused_moe_mxfp4" in lib.moe_last_error()
+    assert lib.moe_workspace_bytes(moe.DTYPE_MXFP4, 64, 1024, 1024, 8, 2, 128) == \
+        lib.moe_workspace_bytes(moe.DTYPE_MXFP8, 64, 1024, 1024, 8, 2, 128)
+
+
 def test_fused_rejects(lib):
     assert _bf16(lib, K=1000) == UNSUPPORTED
     assert _bf16(lib, N=1000) == UNSUPPORTED

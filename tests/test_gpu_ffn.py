@@ -41,9 +41,10 @@ def gpu_forward(sh: W.Shape, inp: dict, block_m: int | None = None, tune=None, r
         x, xs, w1, w2 = (to_dev(inp[n]) for n in ("x", "x_scales", "w1", "w2"))
         s1 = moe.pack_scales_blocked(to_dev(inp["w1_scales"]))
         s2 = moe.pack_scales_blocked(to_dev(inp["w2_scales"]))
+        fwd = moe.fused_moe_mxfp4 if sh.dtype == "mxfp4" else moe.fused_moe_mxfp8
         for _ in range(repeat):
             out = torch.full((sh.T, sh.K), float("nan"), dtype=torch.bfloat16, device="cuda")
-            moe.fused_moe_mxfp8(x, xs, w1, s1, w2, s2, sorted_ids, expert_ids, ntpp, tw, out, bm, tune=tune)
+            fwd(x, xs, w1, s1, w2, s2, sorted_ids, expert_ids, ntpp, tw, out, bm, tune=tune)
             outs.append(out)
     moe.moe_device_status()
     res = [out_bits(o) for o in outs]
@@ -55,9 +56,9 @@ def oracle_forward(sh: W.Shape, inp: dict, tokens=None):
     if sh.dtype == "bf16":
         return oracle.fused_moe_bf16(inp["x"], inp["w1"], inp["w2"], inp["topk_ids"], inp["topk_weights"],
                                      tokens=tokens, unrounded=True)[1]
-    return oracle.fused_moe_mxfp8(inp["x"], inp["x_scales"], inp["w1"], inp["w1_scales"], inp["w2"],
-                                  inp["w2_scales"], inp["topk_ids"], inp["topk_weights"], tokens=tokens,
-                                  unrounded=True)[1]
+    fwd = oracle.fused_moe_mxfp4 if sh.dtype == "mxfp4" else oracle.fused_moe_mxfp8
+    return fwd(inp["x"], inp["x_scales"], inp["w1"], inp["w1_scales"], inp["w2"], inp["w2_scales"],
+               inp["topk_ids"], inp["topk_weights"], tokens=tokens, unrounded=True)[1]
 
 
 def check(sh, got, ref, what):
@@ -87,9 +88,17 @@ SMALL_MXFP8 = [
     small("mxfp8", 300, 256, 256, 16, 4, 128, 1.2),
     small("mxfp8", 12, 1024, 512, 4, 2, 128),     # split-K (4 splits)
 ]
+SMALL_MXFP4 = [                                    # MXFP4 weights, mxfp8 activations
+    small("mxfp4", 200, 256, 512, 8, 2, 128),
+    small("mxfp4", 200, 512, 256, 8, 2, 64),
+    small("mxfp4", 90, 256, 768, 6, 3, 32),
+    small("mxfp4", 300, 256, 256, 16, 4, 128, 1.2),
+    small("mxfp4", 12, 1024, 512, 4, 2, 128),     # split-K
+    small("mxfp4", 1, 256, 256, 3, 1, 16),
+]
 
 
-@pytest.mark.parametrize("sh", SMALL_BF16 + SMALL_MXFP8, ids=lambda s: f"{s.dtype}-T{s.T}-K{s.K}-N{s.N}-E{s.E}-"
+@pytest.mark.parametrize("sh", SMALL_BF16 + SMALL_MXFP8 + SMALL_MXFP4, ids=lambda s: f"{s.dtype}-T{s.T}-K{s.K}-N{s.N}-E{s.E}-"
                          f"k{s.top_k}-bm{s.block_m}")
 def test_small_full_oracle(sh):
     inp = W.inputs(sh, seed=11)
@@ -162,8 +171,9 @@ def _weights(name):
         if sh.dtype == "bf16":
             _WEIGHTS[name] = dict(w1=W.bf16_weights(sh, "w1"), w2=W.bf16_weights(sh, "w2"))
         else:
-            w1, s1 = W.mxfp8_weights(sh, "w1")
-            w2, s2 = W.mxfp8_weights(sh, "w2")
+            wq = W.mxfp4_weights if sh.dtype == "mxfp4" else W.mxfp8_weights
+            w1, s1 = wq(sh, "w1")
+            w2, s2 = wq(sh, "w2")
             _WEIGHTS[name] = dict(w1=w1, w1_scales=s1, w2=w2, w2_scales=s2)
     return _WEIGHTS[name]
 
@@ -182,7 +192,9 @@ def _full_inputs(name, T):
 @pytest.mark.parametrize("name,T,ntok", [("C2", 64, 32), ("C2", 256, 32),
                                          ("C3", 64, 12), ("C3", 256, 12), ("C3", 1024, 12), ("C3", 2048, 12),
                                          ("C3", 4096, 12), ("C3", 8192, 12),
-                                         ("C4", 1024, 6), ("C4", 2048, 6), ("C4", 4096, 6), ("C4", 8192, 6)])
+                                         ("C4", 1024, 6), ("C4", 2048, 6), ("C4", 4096, 6), ("C4", 8192, 6),
+                                         ("C3F4", 64, 12), ("C3F4", 2048, 12), ("C3F4", 8192, 12),
+                                         ("C4F4", 1024, 6), ("C4F4", 8192, 6)])
 def test_full_size_sampled(name, T, ntok):
     """The workload at full size through the GPU path; parity on a seeded token
     sample that includes tokens of the most- and least-loaded experts."""
