@@ -65,7 +65,7 @@ def _load():
         lib.orc_align_capacity.restype = I64
         lib.orc_moe_align.argtypes = [P, I, I, I, I, P, P, P, I64]
         lib.orc_moe_align.restype = I
-        lib.orc_route_topk.argtypes = [P, P, I, I, I, P, P]
+        lib.orc_route_topk.argtypes = [P, P, I, I, I, I, P, P]
         lib.orc_route_topk.restype = I
         lib.orc_pack_scales_bytes.argtypes = [I, I, I]
         lib.orc_pack_scales_bytes.restype = I64
@@ -147,18 +147,21 @@ def moe_align(topk_ids: np.ndarray, E: int, block_m: int, capacity: int | None =
     return sorted_ids, expert_ids, int(ntpp[0])
 
 
-def route_topk(logits: np.ndarray, top_k: int, bias: np.ndarray | None = None):
-    """Router: (T, E) fp32 logits (+ optional (E,) fp32 bias) -> (topk_ids (T, top_k) int32,
-    topk_weights (T, top_k) float64).  Ranking on the fp32 score logits + bias, ties to the
-    lower expert; weights are the renormalised softmax over the kept experts."""
+def route_topk(logits: np.ndarray, top_k: int, bias: np.ndarray | None = None, n_shared: int = 0):
+    """Router: (T, E) fp32 logits (+ optional (E,) fp32 bias) -> (topk_ids (T, top_k + n_shared) int32,
+    topk_weights (T, top_k + n_shared) float64).  Ranking on the fp32 score logits + bias, ties to
+    the lower expert; weights are the renormalised softmax over the kept experts; then n_shared
+    routes to the shared experts E, E+1, ... with weight 1."""
     lg = np.ascontiguousarray(logits, dtype=np.float32)
     T, E = lg.shape
     b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
     if b is not None and b.shape != (E,):
         raise ValueError("bias must have shape (E,)")
-    ids = np.empty((T, top_k), dtype=np.int32)
-    w = np.empty((T, top_k), dtype=np.float64)
-    rc = _load().orc_route_topk(_ptr(lg), None if b is None else _ptr(b), T, E, top_k, _ptr(ids), _ptr(w))
+    kk = top_k + n_shared
+    ids = np.empty((T, kk), dtype=np.int32)
+    w = np.empty((T, kk), dtype=np.float64)
+    rc = _load().orc_route_topk(_ptr(lg), None if b is None else _ptr(b), T, E, top_k, n_shared, _ptr(ids),
+                                _ptr(w))
     if rc != 0:
         raise RuntimeError(f"oracle route_topk failed ({rc})")
     return ids, w

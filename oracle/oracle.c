@@ -210,11 +210,19 @@ int orc_moe_align(const int32_t* topk_ids, int T, int top_k, int E, int block_m,
 /*    in double (the full softmax denominator cancels in the              */
 /*    renormalisation), evaluated as exp(z_j - z_max) for range.          */
 /* Scores must be finite.                                                 */
+/* Shared experts (n_shared >= 0) follow the routed ones: every token     */
+/* gets n_shared more routes, to experts E .. E+n_shared-1, weight 1 --   */
+/* reading: a shared expert processes every token and its output is added */
+/* to the routed sum (the pages name shared experts beside routed ones in */
+/* the fused megakernels of the sgl DeepGEMM PR and DeepGEMM #411 without */
+/* further definition).  Row t of the outputs holds top_k + n_shared      */
+/* entries.                                                               */
 /* ====================================================================== */
 
-int orc_route_topk(const float* logits, const float* bias, int T, int E, int top_k,
+int orc_route_topk(const float* logits, const float* bias, int T, int E, int top_k, int n_shared,
                    int32_t* topk_ids, double* topk_weights) {
-  if (T < 0 || E < 1 || top_k < 1 || top_k > E) return -1;
+  if (T < 0 || E < 1 || top_k < 1 || top_k > E || n_shared < 0) return -1;
+  const int kk = top_k + n_shared;
   float* z = (float*)malloc((size_t)E * sizeof(float));
   unsigned char* taken = (unsigned char*)malloc((size_t)E);
   if (!z || !taken) { free(z); free(taken); return -1; }
@@ -224,8 +232,8 @@ int orc_route_topk(const float* logits, const float* bias, int T, int E, int top
       z[e] = logits[(int64_t)t * E + e] + b; /* one fp32 addition */
       taken[e] = 0;
     }
-    int32_t* ids = topk_ids + (int64_t)t * top_k;
-    double* w = topk_weights + (int64_t)t * top_k;
+    int32_t* ids = topk_ids + (int64_t)t * kk;
+    double* w = topk_weights + (int64_t)t * kk;
     /* selection: repeatedly the largest remaining score, lowest index first */
     for (int j = 0; j < top_k; ++j) {
       int best = -1;
@@ -244,6 +252,10 @@ int orc_route_topk(const float* logits, const float* bias, int T, int E, int top
       sum += w[j];
     }
     for (int j = 0; j < top_k; ++j) w[j] /= sum;
+    for (int j = 0; j < n_shared; ++j) {
+      ids[top_k + j] = E + j;
+      w[top_k + j] = 1.0;
+    }
   }
   free(z);
   free(taken);

@@ -42,8 +42,10 @@ int orc_moe_align(const int32_t* topk_ids, int T, int top_k, int E, int block_m,
 
 /* ---- router (softmax, top-k, renormalisation) -------------------------- */
 /* bias may be NULL.  ids ranked by descending fp32 score logits+bias (ties:
- * lower index); weights in double.  Returns 0, or -1 on bad sizes. */
-int orc_route_topk(const float* logits, const float* bias, int T, int E, int top_k,
+ * lower index); weights in double; then n_shared routes per token to the
+ * shared experts E.. with weight 1 (rows of top_k + n_shared).  Returns 0,
+ * or -1 on bad sizes. */
+int orc_route_topk(const float* logits, const float* bias, int T, int E, int top_k, int n_shared,
                    int32_t* topk_ids, double* topk_weights);
 
 /* ---- blocked weight-scale layout --------------------------------------- */

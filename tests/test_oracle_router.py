@@ -101,3 +101,32 @@ def test_top1_weight_is_one_and_bad_sizes_raise():
     assert ids.tolist() == [[2]] and w.tolist() == [[1.0]]
     with pytest.raises(RuntimeError):
         oracle.route_topk(np.zeros((2, 3), np.float32), 4)
+
+
+def test_shared_experts_append_always_on_routes():
+    rng = np.random.default_rng(10)
+    logits = rng.standard_normal((12, 20)).astype(np.float32)
+    ids0, w0 = oracle.route_topk(logits, 4)
+    ids, w = oracle.route_topk(logits, 4, n_shared=2)
+    assert ids.shape == (12, 6) and np.array_equal(ids[:, :4], ids0) and np.array_equal(w[:, :4], w0)
+    assert (ids[:, 4] == 20).all() and (ids[:, 5] == 21).all() and (w[:, 4:] == 1.0).all()
+
+
+def test_shared_expert_output_is_added_to_the_routed_sum():
+    """A shared expert's contribution is its dense SwiGLU FFN with weight 1 (torch float64)."""
+    import torch.nn.functional as F
+    import workloads as W
+
+    T, K, N, E, k = 10, 64, 128, 4, 2
+    rng = np.random.default_rng(11)
+    x = W.f32_to_bf16_bits(rng.standard_normal((T, K)).astype(np.float32))
+    w1 = W.f32_to_bf16_bits((rng.standard_normal((E + 1, N, K)) / np.sqrt(K)).astype(np.float32))
+    w2 = W.f32_to_bf16_bits((rng.standard_normal((E + 1, K, N // 2)) / np.sqrt(N // 2)).astype(np.float32))
+    ids, w = oracle.route_topk(rng.standard_normal((T, E)).astype(np.float32), k, n_shared=1)
+    both = oracle.fused_moe_bf16(x, w1, w2, ids, w.astype(np.float32), unrounded=True)[1]
+    routed = oracle.fused_moe_bf16(x, w1, w2, ids[:, :k].copy(), w[:, :k].astype(np.float32), unrounded=True)[1]
+    t = lambda b: torch.from_numpy(W.bf16_bits_to_f32(b)).double()
+    h = F.linear(t(x), t(w1[E]))
+    a = (F.silu(h[:, :N // 2]) * h[:, N // 2:]).to(torch.float32).to(torch.bfloat16).double()
+    shared = F.linear(a, t(w2[E])).numpy()
+    np.testing.assert_allclose(both, routed + shared, rtol=1e-12, atol=1e-12)
