@@ -23,6 +23,7 @@ path); time is the max over ranks, ``value`` the sum of all ranks' work.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -62,6 +63,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--router", action="store_true",
                     help="start each step from router logits (moe_route_align) instead of routed ids")
+    ap.add_argument("--shared", type=int, default=0,
+                    help="shared experts after the routed ones (every token, weight 1); needs --router")
     ap.add_argument("--stages", type=int, default=0)
     ap.add_argument("--ctas", type=int, default=0)
     ap.add_argument("--flush-l2", action="store_true",
@@ -252,7 +255,8 @@ def run_reference(args):
 class Problem:
     """Device-resident inputs of one workload and one step of the hot path."""
 
-    def __init__(self, sh: W.Shape, inp: dict, dev, stages: int = 0, ctas: int = 0, router: bool = False):
+    def __init__(self, sh: W.Shape, inp: dict, dev, stages: int = 0, ctas: int = 0, router: bool = False,
+                 n_shared: int = 0):
         import torch
 
         import mixture_experts_ffn_planner_b200 as moe
@@ -265,15 +269,16 @@ class Problem:
 
         bm = self.bm = sh.block_m
         self.router = router
+        self.n_shared = n_shared  # shared experts after the sh.E routed ones (router path only)
         if router:
             # the step starts from router logits: moe_route_align writes ids and weights
             self.logits = up(inp["router_logits"])
             self.bias = None if inp["router_bias"] is None else up(inp["router_bias"])
-            self.ids = torch.empty((sh.T, sh.top_k), dtype=torch.int32, device=dev)
-            self.tw = torch.empty((sh.T, sh.top_k), dtype=torch.float32, device=dev)
+            self.ids = torch.empty((sh.T, sh.top_k + n_shared), dtype=torch.int32, device=dev)
+            self.tw = torch.empty((sh.T, sh.top_k + n_shared), dtype=torch.float32, device=dev)
         else:
             self.ids, self.tw = up(inp["topk_ids"]), up(inp["topk_weights"])
-        cap = moe.moe_align_capacity(sh.T, sh.top_k, sh.E, bm)
+        cap = moe.moe_align_capacity(sh.T, sh.top_k + n_shared, sh.E + n_shared, bm)
         self.s_ids = torch.empty(cap, dtype=torch.int32, device=dev)
         self.e_ids = torch.empty((cap + bm - 1) // bm, dtype=torch.int32, device=dev)
         self.ntpp = torch.empty(1, dtype=torch.int32, device=dev)
@@ -288,7 +293,7 @@ class Problem:
             self.s1 = moe.pack_scales_blocked(up(inp["w1_scales"]))
             self.s2 = moe.pack_scales_blocked(up(inp["w2_scales"]))
             dt = moe.DTYPE_MXFP4 if sh.dtype == "mxfp4" else moe.DTYPE_MXFP8
-        self.ws = torch.empty(moe.moe_workspace_bytes(dt, sh.T, sh.K, sh.N, sh.E, sh.top_k, bm),
+        self.ws = torch.empty(moe.moe_workspace_bytes(dt, sh.T, sh.K, sh.N, sh.E + n_shared, sh.top_k + n_shared, bm),
                               dtype=torch.uint8, device=dev)
         self.plain = moe.Tuning(stages, ctas, None)
         self.stages, self.ctas = stages, ctas
@@ -311,7 +316,7 @@ class Problem:
             plan_event.record()
         if self.router:
             self.moe.moe_route_align(self.logits, self.sh.top_k, self.bm, self.bias, self.ids, self.tw, self.s_ids,
-                                     self.e_ids, self.ntpp)
+                                     self.e_ids, self.ntpp, n_shared=self.n_shared)
         else:
             self.moe.moe_align(self.ids, self.sh.E, self.bm, self.s_ids, self.e_ids, self.ntpp)
         self.fused(self.plain if tune is None else tune)
@@ -517,11 +522,25 @@ def run_b200(args):
     peaks, peak_src = load_peaks()
 
     sh = W.shape(args.workload, args.tokens, **({"E": args.experts} if args.experts else {}))
-    inp = W.inputs(sh, seed=args.seed + rank)  # every replica gets its own batch
+    if args.shared and not args.router:
+        raise SystemExit("--shared needs --router (the router appends the shared experts' routes)")
+    if args.shared:
+        # weights of the routed experts followed by the shared ones
+        sh_w = dataclasses.replace(sh, E=sh.E + args.shared, top_k=sh.top_k + args.shared)
+        inp = W.inputs(sh_w, seed=args.seed + rank)
+        # the generator's routing over the routed experts, then the shared routes (cost model and
+        # CPU baseline; the timed step routes from logits on the GPU)
+        ids, tw = W.routing(sh, seed=args.seed + rank)
+        shared_ids = np.broadcast_to(np.arange(sh.E, sh.E + args.shared, dtype=np.int32), (sh.T, args.shared))
+        inp["topk_ids"] = np.ascontiguousarray(np.concatenate([ids, shared_ids], axis=1))
+        inp["topk_weights"] = np.ascontiguousarray(
+            np.concatenate([tw, np.ones((sh.T, args.shared), np.float32)], axis=1))
+    else:
+        inp = W.inputs(sh, seed=args.seed + rank)  # every replica gets its own batch
     if args.router:
         inp["router_logits"], inp["router_bias"] = W.router_logits(sh, seed=args.seed + rank)
-    cm = cost_model(sh, inp["topk_ids"], peaks)
-    prob = Problem(sh, inp, dev, args.stages, args.ctas, router=args.router)
+    cm = cost_model(sh_w if args.shared else sh, inp["topk_ids"], peaks)
+    prob = Problem(sh, inp, dev, args.stages, args.ctas, router=args.router, n_shared=args.shared)
     flush = args.flush_l2 or cm["bytes_w"] < 4 * 126e6
     m = measure(prob, args.steps, args.warmup, flush_l2=flush, barrier=barrier, local=local)
 
@@ -529,6 +548,8 @@ def run_b200(args):
     line = result_line(sh, cm, m, world, args.steps, args.warmup, peaks, peak_src, flush)
     if args.router:
         line["config"]["router"] = "in the step: moe_route_align (softmax, top-k, renormalise) from fp32 logits"
+    if args.shared:
+        line["config"]["shared_experts"] = args.shared
     if not args.no_e2e:
         ems, h2d, d2h = measure_e2e(prob, args.steps, barrier)
         ems = max_over_ranks(ems, world, dist, dev)

@@ -107,18 +107,29 @@ MOE_API int moe_align(const int32_t* topk_ids, int T, int top_k, int E, int bloc
  *
  *   logits              (T, E) fp32, device, row major, read only; finite.
  *   bias                (E) fp32, device, or NULL for none.
- *   topk_ids            (T, top_k) int32, device, written: kept experts in
- *                       rank order.
- *   topk_weights        (T, top_k) fp32, device, written; each row sums to 1.
+ *   n_shared            shared experts (>= 0): every token also routes to
+ *                       experts E .. E+n_shared-1 with weight 1 (reading: a
+ *                       shared expert processes every token and its output
+ *                       is added to the routed sum).  The FFN then runs with
+ *                       E + n_shared experts (the shared ones stored after
+ *                       the routed ones in w1/w2) and top_k + n_shared
+ *                       routes per token, in the same fused kernels.
+ *   topk_ids            (T, top_k + n_shared) int32, device, written: kept
+ *                       experts in rank order, then the shared experts.
+ *   topk_weights        (T, top_k + n_shared) fp32, device, written; the
+ *                       routed part of each row sums to 1, shared entries 1.
  *   sorted_token_ids, expert_ids, num_tokens_post_padded, capacity: as for
- *                       moe_align (the same bits moe_align gives on topk_ids).
+ *                       moe_align on topk_ids with E + n_shared experts
+ *                       (capacity >= moe_align_capacity(T, top_k + n_shared,
+ *                       E + n_shared, block_m)).
  * Batches of at most 32 tokens are routed inside the planner's CTA; larger
  * ones by an all-SM router kernel chained to the planner.
- * Constraints: as moe_align, plus 1 <= top_k <= min(8, E).  Returns
+ * Constraints: as moe_align, plus 1 <= top_k <= min(8, E), top_k + n_shared
+ * <= 32 and E + n_shared <= 1024.  Returns
  * MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG before any launch otherwise.
  * ---------------------------------------------------------------------- */
-MOE_API int moe_route_align(const float* logits, const float* bias, int T, int E, int top_k, int block_m,
-                    int32_t* topk_ids, float* topk_weights, int32_t* sorted_token_ids,
+MOE_API int moe_route_align(const float* logits, const float* bias, int T, int E, int top_k, int n_shared,
+                    int block_m, int32_t* topk_ids, float* topk_weights, int32_t* sorted_token_ids,
                     int32_t* expert_ids, int32_t* num_tokens_post_padded, int64_t capacity,
                     moe_stream_t stream);
 

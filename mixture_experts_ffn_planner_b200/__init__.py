@@ -85,7 +85,7 @@ _SIGS = {
     "moe_device_status": ([_P], _I),
     "moe_align_capacity": ([_I, _I, _I, _I], _I64),
     "moe_align": ([_P, _I, _I, _I, _I, _P, _P, _P, _I64, _P], _I),
-    "moe_route_align": ([_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I64, _P], _I),
+    "moe_route_align": ([_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I64, _P], _I),
     "pack_scales_blocked_bytes": ([_I, _I, _I], _I64),
     "pack_scales_blocked": ([_P, _P, _I, _I, _I, _P], _I),
     "moe_workspace_bytes": ([_I, _I, _I, _I, _I, _I, _I], _I64),
@@ -197,9 +197,11 @@ def moe_align(topk_ids, E: int, block_m: int, sorted_token_ids=None, expert_ids=
 
 
 def moe_route_align(logits, top_k: int, block_m: int, bias=None, topk_ids=None, topk_weights=None,
-                    sorted_token_ids=None, expert_ids=None, num_tokens_post_padded=None, stream=None):
-    """Router + planner.  logits (T, E) fp32, bias (E,) fp32 or None.  Returns (topk_ids,
-    topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded)."""
+                    sorted_token_ids=None, expert_ids=None, num_tokens_post_padded=None, stream=None,
+                    n_shared: int = 0):
+    """Router + planner.  logits (T, E) fp32, bias (E,) fp32 or None; n_shared shared experts
+    (indices E.., weight 1) follow the routed ones.  Returns (topk_ids, topk_weights,
+    sorted_token_ids, expert_ids, num_tokens_post_padded), the first two (T, top_k + n_shared)."""
     import torch
 
     _need(logits, "logits", (torch.float32,))
@@ -208,14 +210,15 @@ def moe_route_align(logits, top_k: int, block_m: int, bias=None, topk_ids=None, 
         _need(bias, "bias", (torch.float32,))
         if bias.numel() != E:
             raise ValueError("bias must hold E values")
-    cap = moe_align_capacity(T, top_k, E, block_m)
+    kk = top_k + n_shared
+    cap = moe_align_capacity(T, kk, E + n_shared, block_m)
     if cap < 0:
         raise MoeError(-1, "moe_route_align: invalid sizes")
     dev = logits.device
     if topk_ids is None:
-        topk_ids = torch.empty((T, top_k), dtype=torch.int32, device=dev)
+        topk_ids = torch.empty((T, kk), dtype=torch.int32, device=dev)
     if topk_weights is None:
-        topk_weights = torch.empty((T, top_k), dtype=torch.float32, device=dev)
+        topk_weights = torch.empty((T, kk), dtype=torch.float32, device=dev)
     if sorted_token_ids is None:
         sorted_token_ids = torch.empty(cap, dtype=torch.int32, device=dev)
     if expert_ids is None:
@@ -225,14 +228,14 @@ def moe_route_align(logits, top_k: int, block_m: int, bias=None, topk_ids=None, 
         num_tokens_post_padded = torch.empty(1, dtype=torch.int32, device=dev)
     _need(topk_ids, "topk_ids", (torch.int32,))
     _need(topk_weights, "topk_weights", (torch.float32,))
-    if topk_ids.numel() < T * top_k or topk_weights.numel() < T * top_k:
-        raise ValueError("topk_ids / topk_weights must hold T * top_k entries")
+    if topk_ids.numel() < T * kk or topk_weights.numel() < T * kk:
+        raise ValueError("topk_ids / topk_weights must hold T * (top_k + n_shared) entries")
     for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
                  (num_tokens_post_padded, "num_tokens_post_padded")):
         _need(t, n, (torch.int32,))
     if expert_ids.numel() < (sorted_token_ids.numel() + block_m - 1) // block_m:
         raise ValueError("expert_ids must hold ceil(capacity / block_m) entries")
-    _check(load().moe_route_align(_ptr(logits), _ptr(bias), T, E, top_k, block_m, _ptr(topk_ids),
+    _check(load().moe_route_align(_ptr(logits), _ptr(bias), T, E, top_k, n_shared, block_m, _ptr(topk_ids),
                                   _ptr(topk_weights), _ptr(sorted_token_ids), _ptr(expert_ids),
                                   _ptr(num_tokens_post_padded), sorted_token_ids.numel(), _stream(stream)))
     return topk_ids, topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded

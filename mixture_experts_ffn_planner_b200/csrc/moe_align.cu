@@ -89,15 +89,24 @@ constexpr int kRouteMaxK = 8;
 // measured faster from two tokens per warp on.
 constexpr int kRouteFusedMaxTokens = 32;
 
+// Shared experts follow the routed ones: with n_shared > 0 every token also
+// routes, with weight 1, to experts E .. E+n_shared-1 (reading: a shared
+// expert processes every token and its output is added to the routed sum;
+// the fused megakernels of the sgl DeepGEMM PR and DeepGEMM #411 run shared
+// experts beside the routed ones).  Their GEMMs then run as ordinary,
+// densely filled units of the same fused kernels.
+//
 // One warp routes token t.  Lane l scans experts l, l+32, ... keeping its
 // best kRouteMaxK in a sorted register list (compare-and-swap down a fixed
 // list, so equal scores keep the earlier, lower index ahead); k rounds of a
 // warp-wide arg-max (ties to the lower index) then merge the 32 lists.  Lane
-// j < k ends with the j-th expert and its weight, written to the outputs and,
-// when ids16 is given, to the staged id array at position t*k + j - id0.
+// j < k ends with the j-th expert and its weight, lane k + s with shared
+// expert E + s; row t of the outputs holds k + n_shared entries, also written
+// to the staged id array (when ids16 is given) at t*(k + n_shared) + j - id0.
 __device__ __forceinline__ void route_token(const float* __restrict__ logits, const float* __restrict__ bias,
-                                            int t, int E, int k, int lane, int32_t* __restrict__ topk_ids,
-                                            float* __restrict__ topk_w, uint16_t* ids16, int id0) {
+                                            int t, int E, int k, int n_shared, int lane,
+                                            int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
+                                            uint16_t* ids16, int id0) {
   float lv[kRouteMaxK];
   int le[kRouteMaxK];
 #pragma unroll
@@ -154,11 +163,13 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits, co
   float sum = w;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-  if (lane < k) {
-    const int64_t r = static_cast<int64_t>(t) * k + lane;
-    topk_ids[r] = my_e;
-    topk_w[r] = w / sum;
-    if (ids16) ids16[r - id0] = static_cast<uint16_t>(my_e);
+  const int kk = k + n_shared;
+  if (lane < kk) {
+    const int64_t r = static_cast<int64_t>(t) * kk + lane;
+    const int e = lane < k ? my_e : E + (lane - k);
+    topk_ids[r] = e;
+    topk_w[r] = lane < k ? w / sum : 1.0f;
+    if (ids16) ids16[r - id0] = static_cast<uint16_t>(e);
   }
 }
 
@@ -166,12 +177,13 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits, co
 // planner that follows is chained by programmatic dependent launch.
 __global__ void __launch_bounds__(256) moe_route_kernel(const float* __restrict__ logits,
                                                         const float* __restrict__ bias, int T, int E, int k,
-                                                        int32_t* __restrict__ topk_ids,
+                                                        int n_shared, int32_t* __restrict__ topk_ids,
                                                         float* __restrict__ topk_w) {
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, nw = (gridDim.x * blockDim.x) >> 5;
-  for (int t = gw; t < T; t += nw) route_token(logits, bias, t, E, k, lane, topk_ids, topk_w, nullptr, 0);
+  for (int t = gw; t < T; t += nw)
+    route_token(logits, bias, t, E, k, n_shared, lane, topk_ids, topk_w, nullptr, 0);
 }
 
 // Planner.  With route_T > 0 (one CTA, at most one token per warp) the CTA first
@@ -182,7 +194,7 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
                      int32_t* __restrict__ sorted_ids, int32_t* __restrict__ expert_ids,
                      int32_t* __restrict__ ntpp_out, int64_t capacity, int staged,
                      const float* __restrict__ logits, const float* __restrict__ bias, int route_T, int route_k,
-                     int32_t* route_ids, float* __restrict__ route_w) {
+                     int route_shared, int32_t* route_ids, float* __restrict__ route_w) {
   extern __shared__ int32_t sm[];
   int32_t* hist = sm;                         // [kAlignWarps][E], later start offsets
   int32_t* cnt = hist + kAlignWarps * E;      // [E] this CTA's count per expert
@@ -204,7 +216,7 @@ __global__ void __launch_bounds__(kAlignThreads, 1)
   //    produces them instead.
   if (route_T > 0) {
     for (int t = warp; t < route_T; t += kAlignWarps)
-      route_token(logits, bias, t, E, route_k, lane, route_ids, route_w, ids16, 0);
+      route_token(logits, bias, t, E - route_shared, route_k, route_shared, lane, route_ids, route_w, ids16, 0);
   } else if (staged) {
 #pragma unroll 4
     for (int i = clo + tid; i < chi; i += kAlignThreads) {
@@ -342,8 +354,8 @@ extern "C" int64_t moe_align_capacity(int T, int top_k, int E, int block_m) {
 // after_router chains the launch to a preceding router kernel.
 static int launch_align(const int32_t* topk_ids, int T, int top_k, int E, int block_m, int32_t* sorted_token_ids,
                         int32_t* expert_ids, int32_t* num_tokens_post_padded, int64_t capacity, moe_stream_t stream,
-                        const float* logits, const float* bias, int route_T, int32_t* route_ids, float* route_w,
-                        bool after_router) {
+                        const float* logits, const float* bias, int route_T, int route_k, int route_shared,
+                        int32_t* route_ids, float* route_w, bool after_router) {
   const int R = T * top_k;
   const int csize = R >= kAlignClusterMinIds ? kAlignClusterMax : 1;
   const int cchunk = (R + csize - 1) / csize;
@@ -378,7 +390,7 @@ static int launch_align(const int32_t* topk_ids, int T, int top_k, int E, int bl
   cfg.numAttrs = after_router ? 2 : 1;
   const cudaError_t lerr = cudaLaunchKernelEx(&cfg, moe_align_kernel, topk_ids, R, E, block_m, sorted_token_ids,
                                               expert_ids, num_tokens_post_padded, capacity, staged, logits, bias,
-                                              route_T, top_k, route_ids, route_w);
+                                              route_T, route_k, route_shared, route_ids, route_w);
   if (lerr != cudaSuccess) return cuda_fail("moe_align: launch", lerr);
   const cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return cuda_fail("moe_align: launch", err);
@@ -404,11 +416,11 @@ extern "C" int moe_align(const int32_t* topk_ids, int T, int top_k, int E, int b
     return fail(MOE_ERR_INVALID_ARG, "moe_align: null pointer");
 
   return launch_align(topk_ids, T, top_k, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded, capacity,
-                      stream, nullptr, nullptr, 0, nullptr, nullptr, false);
+                      stream, nullptr, nullptr, 0, 0, 0, nullptr, nullptr, false);
 }
 
-extern "C" int moe_route_align(const float* logits, const float* bias, int T, int E, int top_k, int block_m,
-                               int32_t* topk_ids, float* topk_weights, int32_t* sorted_token_ids,
+extern "C" int moe_route_align(const float* logits, const float* bias, int T, int E, int top_k, int n_shared,
+                               int block_m, int32_t* topk_ids, float* topk_weights, int32_t* sorted_token_ids,
                                int32_t* expert_ids, int32_t* num_tokens_post_padded, int64_t capacity,
                                moe_stream_t stream) {
   if (T < 0) return fail(MOE_ERR_INVALID_ARG, "moe_route_align: need T >= 0");
@@ -416,11 +428,15 @@ extern "C" int moe_route_align(const float* logits, const float* bias, int T, in
     return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: E must be in [1, %d], got %d", kMaxExperts, E);
   if (top_k < 1 || top_k > kRouteMaxK || top_k > E)
     return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: top_k must be in [1, min(%d, E)], got %d", kRouteMaxK, top_k);
+  if (n_shared < 0 || top_k + n_shared > 32 || E + n_shared > kMaxExperts)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_route_align: need n_shared >= 0, top_k + n_shared <= 32 and E + n_shared <= %d", kMaxExperts);
+  const int kk = top_k + n_shared, Et = E + n_shared;  // the planner sees the shared routes as ordinary ones
   if (!valid_block_m(block_m))
     return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: block_m must be 16, 32, 64 or 128, got %d", block_m);
-  const int64_t need = moe_align_capacity(T, top_k, E, block_m);
+  const int64_t need = moe_align_capacity(T, kk, Et, block_m);
   if (need >= (int64_t(1) << 31))
-    return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: T*top_k + E*(block_m-1) must be < 2^31");
+    return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: T*(top_k+n_shared) + (E+n_shared)*(block_m-1) must be < 2^31");
   if (capacity < need)
     return fail(MOE_ERR_INVALID_ARG, "moe_route_align: capacity %lld < required %lld", (long long)capacity,
                 (long long)need);
@@ -432,11 +448,11 @@ extern "C" int moe_route_align(const float* logits, const float* bias, int T, in
   const bool fused = T <= kRouteFusedMaxTokens;
   if (!fused && T > 0) {
     const int blocks = std::min<int64_t>((static_cast<int64_t>(T) + 7) / 8, static_cast<int64_t>(sm_count()) * 8);
-    moe_route_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(logits, bias, T, E, top_k,
+    moe_route_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(logits, bias, T, E, top_k, n_shared,
                                                                                topk_ids, topk_weights);
     const cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return cuda_fail("moe_route_align: router launch", err);
   }
-  return launch_align(topk_ids, T, top_k, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded, capacity,
-                      stream, logits, bias, fused ? T : 0, topk_ids, topk_weights, !fused && T > 0);
+  return launch_align(topk_ids, T, kk, Et, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded, capacity,
+                      stream, logits, bias, fused ? T : 0, top_k, n_shared, topk_ids, topk_weights, !fused && T > 0);
 }

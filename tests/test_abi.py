@@ -66,9 +66,9 @@ def test_moe_align_rejects(lib):
     assert b"block_m" in lib.moe_last_error() or True
 
 
-def _route(lib, T=4, E=8, k=2, bm=64, cap=None, ptrs=(8, 8, 8, 8, 8, 8, 8), bias=None):
-    cap = lib.moe_align_capacity(T, k, E, bm) if cap is None else cap
-    return lib.moe_route_align(ptrs[0], bias, T, E, k, bm, ptrs[1], ptrs[2], ptrs[3], ptrs[4], ptrs[5], cap, None)
+def _route(lib, T=4, E=8, k=2, bm=64, cap=None, ptrs=(8, 8, 8, 8, 8, 8, 8), bias=None, S=0):
+    cap = lib.moe_align_capacity(T, k + S, E + S, bm) if cap is None else cap
+    return lib.moe_route_align(ptrs[0], bias, T, E, k, S, bm, ptrs[1], ptrs[2], ptrs[3], ptrs[4], ptrs[5], cap, None)
 
 
 def test_moe_route_align_rejects(lib):
@@ -83,6 +83,10 @@ def test_moe_route_align_rejects(lib):
     assert _route(lib, ptrs=(8, 0, 8, 8, 8, 8, 8)) == INVALID   # topk_ids
     assert _route(lib, ptrs=(8, 8, 0, 8, 8, 8, 8)) == INVALID   # topk_weights
     assert _route(lib, ptrs=(8, 8, 8, 0, 8, 8, 8)) == INVALID   # sorted_token_ids
+    assert _route(lib, S=-1) == UNSUPPORTED
+    assert _route(lib, k=8, E=64, S=25) == UNSUPPORTED       # more than 32 routes per token
+    assert _route(lib, E=1020, S=5) == UNSUPPORTED           # more than 1024 experts with the shared ones
+    assert _route(lib, S=2, cap=lib.moe_align_capacity(4, 2, 8, 64)) == INVALID  # capacity without the shared
     assert b"moe_route_align" in lib.moe_last_error()
 
 

@@ -21,32 +21,32 @@ pytestmark = pytest.mark.gpu
 W_TOL = 2e-6
 
 
-def _run(logits: np.ndarray, bias, k: int, bm: int):
+def _run(logits: np.ndarray, bias, k: int, bm: int, S: int = 0):
     import torch
     import mixture_experts_ffn_planner_b200 as moe
 
     T, E = logits.shape
-    cap = moe.moe_align_capacity(T, k, E, bm)
+    cap = moe.moe_align_capacity(T, k + S, E + S, bm)
     d_logits = to_dev(logits) if logits.size else torch.empty((T, E), dtype=torch.float32, device="cuda")
     d_bias = None if bias is None else to_dev(bias)
     # poisoned outputs: any element the kernels skip shows up
-    ids = torch.full((T, k), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
-    w = torch.full((T, k), float("nan"), dtype=torch.float32, device="cuda")
+    ids = torch.full((T, k + S), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
+    w = torch.full((T, k + S), float("nan"), dtype=torch.float32, device="cuda")
     s = torch.full((cap,), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
     e = torch.full(((cap + bm - 1) // bm,), 0x5A5A5A5A, dtype=torch.int32, device="cuda")
     n = torch.full((1,), -7, dtype=torch.int32, device="cuda")
-    moe.moe_route_align(d_logits, k, bm, d_bias, ids, w, s, e, n)
+    moe.moe_route_align(d_logits, k, bm, d_bias, ids, w, s, e, n, n_shared=S)
     torch.cuda.synchronize()
     return ids.cpu().numpy(), w.cpu().numpy(), s.cpu().numpy(), e.cpu().numpy(), int(n.cpu().numpy()[0])
 
 
-def _check(logits, bias, k, bm):
+def _check(logits, bias, k, bm, S=0):
     T, E = logits.shape
-    rid, rw = oracle.route_topk(logits, k, bias)
-    gid, gw, gs, ge, gn = _run(logits, bias, k, bm)
+    rid, rw = oracle.route_topk(logits, k, bias, n_shared=S)
+    gid, gw, gs, ge, gn = _run(logits, bias, k, bm, S)
     np.testing.assert_array_equal(gid, rid)
     assert np.all(np.abs(gw.astype(np.float64) - rw) <= W_TOL), float(np.max(np.abs(gw - rw)))
-    rs, re_, rn = oracle.moe_align(rid, E, bm)
+    rs, re_, rn = oracle.moe_align(rid, E + S, bm)
     assert gn == rn
     np.testing.assert_array_equal(gs, rs)
     np.testing.assert_array_equal(ge, re_)
@@ -99,3 +99,45 @@ def test_routed_ids_drive_the_ffn():
     rid, rw = oracle.route_topk(logits, sh.top_k, bias)
     ref = oracle.fused_moe_bf16(inp["x"], inp["w1"], inp["w2"], rid, rw.astype(np.float32), unrounded=True)[1]
     assert_bf16_parity(got, ref, "routed C1")
+
+
+@pytest.mark.parametrize("T", [8, 32, 300])
+@pytest.mark.parametrize("S", [1, 2])
+def test_shared_experts(T, S):
+    rng = np.random.default_rng(T * 7 + S)
+    _check(rng.standard_normal((T, 64)).astype(np.float32), None, 6, 64, S)
+    sh = W.shape("C3", 64)
+    logits, bias = W.router_logits(sh)
+    _check(logits[:T] if T <= 64 else np.tile(logits, (5, 1))[:T], bias, sh.top_k, sh.block_m, S)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "mxfp8"])
+def test_shared_expert_in_the_fused_kernels(dtype):
+    """Routed experts plus one shared expert (stored after them) in one fused call, against
+    the oracle routing with its own router and running the FFN on E + 1 experts."""
+    import torch
+    import mixture_experts_ffn_planner_b200 as moe
+    from tests.helpers import assert_bf16_parity, assert_mxfp8_parity, out_bits
+
+    E, S, k, T, K, N, bm = 8, 1, 2, 200, 256, 512, 64
+    sh = W.Shape(name="S", dtype=dtype, T=T, K=K, N=N, E=E + S, top_k=k + S, block_m=bm, zipf_s=None)
+    inp = W.inputs(sh, seed=5)                  # x and the weights of E + S experts
+    logits = np.random.default_rng(6).standard_normal((T, E)).astype(np.float32)
+    _, d_w, s_ids, e_ids, ntpp = moe.moe_route_align(to_dev(logits), k, bm, None, n_shared=S)
+    out = torch.full((T, K), float("nan"), dtype=torch.bfloat16, device="cuda")
+    rid, rw = oracle.route_topk(logits, k, None, n_shared=S)
+    if dtype == "bf16":
+        x, w1, w2 = (to_dev(inp[n], torch.bfloat16) for n in ("x", "w1", "w2"))
+        moe.fused_moe_bf16(x, w1, w2, s_ids, e_ids, ntpp, d_w, out, bm)
+        ref = oracle.fused_moe_bf16(inp["x"], inp["w1"], inp["w2"], rid, rw.astype(np.float32), unrounded=True)[1]
+        check = assert_bf16_parity
+    else:
+        x, xs, w1, w2 = (to_dev(inp[n]) for n in ("x", "x_scales", "w1", "w2"))
+        s1 = moe.pack_scales_blocked(to_dev(inp["w1_scales"]))
+        s2 = moe.pack_scales_blocked(to_dev(inp["w2_scales"]))
+        moe.fused_moe_mxfp8(x, xs, w1, s1, w2, s2, s_ids, e_ids, ntpp, d_w, out, bm)
+        ref = oracle.fused_moe_mxfp8(inp["x"], inp["x_scales"], inp["w1"], inp["w1_scales"], inp["w2"],
+                                     inp["w2_scales"], rid, rw.astype(np.float32), unrounded=True)[1]
+        check = assert_mxfp8_parity
+    moe.moe_device_status()
+    check(out_bits(out), ref, f"{dtype} with a shared expert")
