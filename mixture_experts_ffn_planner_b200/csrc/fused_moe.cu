@@ -1,4 +1,5 @@
-// Fused MoE expert-FFN forward for sm_100a (bf16 and mxfp8 paths).
+// Fused MoE expert-FFN forward for sm_100a (bf16 and mxfp8 paths; the mxfp8
+// path also takes MXFP4 weights).
 //
 // What is computed -- "Prime Flash MoE: Fused MoE Kernels for Blackwell",
 // intro / API / Shapes, and "[RFC] Fused W8A8 MoE megakernel on H20",
@@ -24,9 +25,13 @@
 //            on mxfp8, their scales; completion is tracked by the stage's
 //            mbarrier, so the gather warps never wait on their own copies),
 //            6-13 epilogue (two warps per TMEM lane quadrant, one per column
-//            half).
+//            half).  When the units cannot fill the SMs (decode-sized
+//            problems), a unit's K range is split over several CTAs and the
+//            fp32 partial accumulators are summed, in split order, by
+//   reduce   a small kernel that applies SwiGLU (and the requant) to the sum.
 //   phase 2  persistent kernel, unit = (block b, 256 output features).  A =
-//            the block's intermediate rows (TMA), B = 256 rows of w2[e] (TMA),
+//            the block's intermediate rows (TMA, one 128-row box for blocks of
+//            at least 64 rows), B = 256 rows of w2[e] (TMA, one box),
 //            D in TMEM; each epilogue thread scales its row by the routing
 //            weight and writes one row segment per route (fp32 on the bf16
 //            path; bf16 on the mxfp8 path, whose tolerance leaves room for
@@ -34,7 +39,10 @@
 //   combine  out[t] = bf16(sum over the token's routes, in route order), a
 //            deterministic HBM-bound pass.
 // The weight tiles are streamed once per unit through a multi-stage shared
-// memory ring by TMA; the weights are the dominant HBM traffic.
+// memory ring by TMA; the weights are the dominant HBM traffic.  MXFP4
+// weights (e2m1, two per byte) are expanded by the copy itself into the
+// unpacked shared-memory form the block-scaled MMA reads, so the two GEMM
+// kernels differ only in byte counts and the MMA's B format.
 #include <algorithm>
 #include <mutex>
 
@@ -1365,7 +1373,7 @@ static int run_fused(const FusedArgs& a) {
     if ((rc = set_smem_attr(moe_p1_kernel<false>, smem1, attr_done[2])) != MOE_OK) return rc;
     if ((rc = set_smem_attr(moe_p2_kernel<false>, smem2, attr_done[3])) != MOE_OK) return rc;
   }
-  // The three launches are chained by programmatic dependent launch: each
+  // The four launches are chained by programmatic dependent launch: each
   // kernel lets the next one be scheduled early (prologue: barriers, TMEM,
   // tensor-map prefetch) and the next one waits (griddepcontrol.wait) before
   // reading the previous one's results.
