@@ -16,6 +16,9 @@ phase, timed with CUDA events recorded by the library on the launching
 stream), the end-to-end figure through host buffers, SM clocks sampled during
 the timed region, and the CPU oracle timed on a bounded token sample.
 
+Other rows: ``--workload C3F4`` / ``C4F4`` run the MXFP4-weight path; ``--router`` starts each step
+from router logits (``moe_route_align``); ``--router --shared S`` adds S shared experts.
+
 Multi-GPU: ``torchrun --nproc-per-node N bench.py --gpus N``; every rank is an
 independent replica with all experts resident (no collective on the data
 path); time is the max over ranks, ``value`` the sum of all ranks' work.
@@ -69,7 +72,12 @@ def parse_args(argv=None):
     ap.add_argument("--ctas", type=int, default=0)
     ap.add_argument("--flush-l2", action="store_true",
                     help="flush L2 between steps (automatic when the touched weights are < 4x L2)")
-    return ap.parse_args(argv)
+    args = ap.parse_args(argv)
+    if args.shared and not args.router:
+        ap.error("--shared needs --router (the router appends the shared experts' routes)")
+    if args.shared < 0:
+        ap.error("--shared must be >= 0")
+    return args
 
 
 def load_peaks():
@@ -522,8 +530,6 @@ def run_b200(args):
     peaks, peak_src = load_peaks()
 
     sh = W.shape(args.workload, args.tokens, **({"E": args.experts} if args.experts else {}))
-    if args.shared and not args.router:
-        raise SystemExit("--shared needs --router (the router appends the shared experts' routes)")
     if args.shared:
         # weights of the routed experts followed by the shared ones
         sh_w = dataclasses.replace(sh, E=sh.E + args.shared, top_k=sh.top_k + args.shared)
