@@ -1,4 +1,5 @@
 // Error reporting and device queries shared by every entry point.
+#include <atomic>
 #include <stdarg.h>
 #include <stdio.h>
 
@@ -22,13 +23,17 @@ int cuda_fail(const char* what, cudaError_t err) {
 }
 
 int sm_count() {
-  static int cached[kMaxDevices] = {};
+  // per-device cache; host threads may race to fill it, always with the same value
+  static std::atomic<int> cached[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev < kMaxDevices && cached[dev] > 0) return cached[dev];
+  if (dev < kMaxDevices) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  if (dev < kMaxDevices) cached[dev] = n;
+  if (dev < kMaxDevices) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 

@@ -44,6 +44,7 @@
 // unpacked shared-memory form the block-scaled MMA reads, so the two GEMM
 // kernels differ only in byte counts and the MMA's B format.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -1180,15 +1181,17 @@ static int make_tmap(CUtensorMap* m, const void* base, TmapKind kind, int64_t ro
 
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// done[dev]: the attribute is set on that device (host threads may race to
+// set it; setting it twice is harmless)
 template <typename K>
-static int set_smem_attr(K kernel, int bytes, bool* done) {
+static int set_smem_attr(K kernel, int bytes, std::atomic<bool>* done) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice");
-  if (dev < kMaxDevices && done[dev]) return MOE_OK;
+  if (dev < kMaxDevices && done[dev].load(std::memory_order_relaxed)) return MOE_OK;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit) != cudaSuccess)
     return cuda_fail("cudaFuncSetAttribute");
   (void)bytes;
-  if (dev < kMaxDevices) done[dev] = true;
+  if (dev < kMaxDevices) done[dev].store(true, std::memory_order_relaxed);
   return MOE_OK;
 }
 
@@ -1268,14 +1271,16 @@ static int run_fused(const FusedArgs& a) {
 
   const int I = a.N / 2;
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
-  static int* status_ptr[kMaxDevices] = {};
+  static std::atomic<int*> status_ptr[kMaxDevices];  // per device; races store the same address
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice");
   if (dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "%s: device index %d too large", nm, dev);
-  if (!status_ptr[dev]) {
+  int* status = status_ptr[dev].load(std::memory_order_relaxed);
+  if (!status) {
     void* sp = nullptr;
     if (cudaGetSymbolAddress(&sp, g_moe_status) != cudaSuccess) return cuda_fail("cudaGetSymbolAddress");
-    status_ptr[dev] = static_cast<int*>(sp);
+    status = static_cast<int*>(sp);
+    status_ptr[dev].store(status, std::memory_order_relaxed);
   }
 
   CUtensorMap tm_w1, tm_w2, tm_w2x, tm_act, tm_actx;
@@ -1312,7 +1317,7 @@ static int run_fused(const FusedArgs& a) {
   p1.act_sf = ws + L.act_sf;
   p1.flags = reinterpret_cast<int32_t*>(ws + L.flags);
   p1.part = reinterpret_cast<float*>(ws + L.part);
-  p1.status = status_ptr[dev];
+  p1.status = status;
   p1.K = a.K; p1.N = a.N; p1.I = I; p1.E = a.E; p1.top_k = a.top_k; p1.bm = a.bm;
   p1.R = a.T * a.top_k;
   p1.max_blocks = max_blocks;
@@ -1365,7 +1370,7 @@ static int run_fused(const FusedArgs& a) {
       return cuda_fail("fused_moe: cudaEventRecord");
     return MOE_OK;
   };
-  static bool attr_done[4][kMaxDevices] = {};
+  static std::atomic<bool> attr_done[4][kMaxDevices];
   if (a.fp8) {
     if ((rc = set_smem_attr(moe_p1_kernel<true>, smem1, attr_done[0])) != MOE_OK) return rc;
     if ((rc = set_smem_attr(moe_p2_kernel<true>, smem2, attr_done[1])) != MOE_OK) return rc;
@@ -1406,14 +1411,15 @@ static int run_fused(const FusedArgs& a) {
   if (err != cudaSuccess) return cuda_fail("fused_moe: down phase launch", err);
   if ((rc = mark(2)) != MOE_OK) return rc;
   // one full wave of resident blocks (grid-stride beyond it)
-  static int comb_occ[2] = {0, 0};
-  int& occ = comb_occ[a.fp8 ? 1 : 0];
+  static std::atomic<int> comb_occ[2];  // races store the same value
+  int occ = comb_occ[a.fp8 ? 1 : 0].load(std::memory_order_relaxed);
   if (occ == 0) {
     int nb = 0;
     err = a.fp8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<__nv_bfloat16, 8>, 256, 0)
                 : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<float, 8>, 256, 0);
     if (err != cudaSuccess) return cuda_fail("fused_moe: combine occupancy query", err);
     occ = nb < 1 ? 1 : nb;
+    comb_occ[a.fp8 ? 1 : 0].store(occ, std::memory_order_relaxed);
   }
   const int64_t nvec = static_cast<int64_t>(a.T) * (a.K / 8);
   const int64_t cblocks = (nvec + 255) / 256;

@@ -33,6 +33,7 @@
 // and expert_ids is filled block by block; these writes are spread over the
 // cluster's CTAs.
 #include <algorithm>
+#include <atomic>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -367,12 +368,12 @@ static int launch_align(const int32_t* topk_ids, int T, int top_k, int E, int bl
     return fail(MOE_ERR_UNSUPPORTED, "moe_route_align: the in-planner router needs one CTA with staged ids");
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("moe_align: cudaGetDevice");
-  static bool attr_set[kMaxDevices] = {};
-  if (dev < kMaxDevices && !attr_set[dev]) {
+  static std::atomic<bool> attr_set[kMaxDevices];  // per device; setting it twice is harmless
+  if (dev < kMaxDevices && !attr_set[dev].load(std::memory_order_relaxed)) {
     if (cudaFuncSetAttribute(moe_align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAlignSmemLimit) !=
         cudaSuccess)
       return cuda_fail("moe_align: cudaFuncSetAttribute");
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_relaxed);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(csize, 1, 1);
