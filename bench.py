@@ -62,6 +62,8 @@ def parse_args(argv=None):
     ap.add_argument("--experts", type=int, default=0, help="override the workload's expert count (profiling)")
     ap.add_argument("--seed", type=int, default=W.DEFAULT_SEED)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU oracle baseline")
+    ap.add_argument("--cpu-threads", type=int, default=0,
+                    help="threads of the CPU oracle (baseline and reference arm); 0 = every host core")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--router", action="store_true",
@@ -77,6 +79,8 @@ def parse_args(argv=None):
         ap.error("--shared needs --router (the router appends the shared experts' routes)")
     if args.shared < 0:
         ap.error("--shared must be >= 0")
+    if args.cpu_threads < 0:
+        ap.error("--cpu-threads must be >= 0")
     return args
 
 
@@ -189,12 +193,14 @@ def kernel_traffic(kernel: str, workload_tag: str):
 
 
 # ----------------------------------------------------------------------------- CPU oracle legs
-def oracle_sample_rate(sh: W.Shape, inp: dict, seconds: float, seed: int):
+def oracle_threads(requested: int) -> int:
+    return requested if requested > 0 else (os.cpu_count() or 1)
+
+
+def oracle_sample_rate(sh: W.Shape, inp: dict, seconds: float, seed: int, threads: int = 0):
     """Times the oracle on a growing token sample until ~`seconds` of work; returns
     (TFLOP/s, threads, description)."""
-    import oracle
-
-    thr = os.cpu_count() or 1
+    thr = oracle_threads(threads)
     n, spent, flops = 1, 0.0, 0.0
     perm = np.random.default_rng(seed).permutation(sh.T)
     used = 0
@@ -229,7 +235,7 @@ def run_reference(args):
         return 0
     sh = W.shape(args.workload, args.tokens, **({"E": args.experts} if args.experts else {}))
     inp = W.inputs(sh, seed=args.seed)
-    thr = os.cpu_count() or 1
+    thr = oracle_threads(args.cpu_threads)
     # calibrate: tokens per step such that all steps fit in ~2 minutes
     t0 = time.perf_counter()
     _run_oracle(sh, inp, np.array([0], np.int32), thr)
@@ -343,6 +349,8 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
     Pass 2 (the per-kernel breakdown): the same steps with the library's phase
     events recorded between its launches (events between launches can keep the
     launches from overlapping, so pass 2 is used for the per-kernel times only).
+    With flush_l2, pass 3 runs the steps back to back without the flush (warm
+    L2), reported beside the cold time and labelled as such.
     """
     import torch
 
@@ -370,10 +378,10 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
         clocks.start()
         time.sleep(0.3)
 
-    def timed(tunes=None, pev=None):
+    def timed(tunes=None, pev=None, cold=flush_l2):
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)] \
-            if flush_l2 else None
+            if cold else None
         t0.record(stream)
         for i in range(steps):
             if s_ev:
@@ -397,7 +405,12 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
     tunes = [moe.Tuning.with_events(e, prob.stages, prob.ctas) for e in ev]
     timed(tunes, pev)
     moe.moe_device_status()
-    return {"total_ms": total_ms, "ms_step": total_ms / steps,
+    warm_ms = None
+    if flush_l2:
+        prob.step()  # the last flush left L2 cold; one untimed step warms it
+        warm_ms = timed(cold=False) / steps
+        moe.moe_device_status()
+    return {"total_ms": total_ms, "ms_step": total_ms / steps, "warm_ms_step": warm_ms,
             "plan_ms": sum(a.elapsed_time(e[0]) for a, e in zip(pev, ev)) / steps,
             "p1_ms": sum(e[0].elapsed_time(e[1]) for e in ev) / steps,
             "p2_ms": sum(e[1].elapsed_time(e[2]) for e in ev) / steps,
@@ -492,6 +505,9 @@ def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
         "roofline": roofline_of_p1(sh, cm, m["p1_ms"], peaks, peak_src),
         "gpu_launches": m["launches"],
         "clocks": m["clocks"],
+        **({"warm": {"us_per_call": m["warm_ms_step"] * 1e3,
+                     "l2": "not flushed: steps back to back, so weights can stay L2-resident (not the reported value)"}}
+           if m.get("warm_ms_step") else {}),
     }
 
 
@@ -563,7 +579,7 @@ def run_b200(args):
                        "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                        "us_per_call": 1e3 * ems / args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, thr, desc, spent = oracle_sample_rate(sh, inp, args.cpu_seconds, args.seed)
+        rate, thr, desc, spent = oracle_sample_rate(sh, inp, args.cpu_seconds, args.seed, args.cpu_threads)
         line["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                                 "sample": desc, "seconds": spent}
     if rank == 0:

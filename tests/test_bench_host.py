@@ -34,3 +34,26 @@ def test_option_checks():
         bench.parse_args(["--router", "--shared", "-1"])
     a = bench.parse_args(["--router", "--shared", "2", "--workload", "C3F4", "--tokens", "64"])
     assert a.router and a.shared == 2 and a.workload == "C3F4"
+
+
+def test_cpu_threads_option():
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--cpu-threads", "-1"])
+    assert bench.oracle_threads(bench.parse_args(["--cpu-threads", "1"]).cpu_threads) == 1
+    assert bench.oracle_threads(0) >= 1
+
+
+def _m(warm):
+    return {"ms_step": 2.0, "warm_ms_step": warm, "plan_ms": 0.01, "p1_ms": 1.2, "p2_ms": 0.7, "cb_ms": 0.05,
+            "clocks": None, "launches": 20}
+
+
+def test_warm_time_is_reported_beside_the_cold_one():
+    sh = W.shape("C1", 64)
+    ids = np.tile(np.arange(sh.top_k, dtype=np.int32), (sh.T, 1))
+    cm = bench.cost_model(sh, ids, PEAKS)
+    cold = bench.result_line(sh, cm, _m(1.5), 1, 4, 3, PEAKS, "measured", True)
+    assert cold["us_per_call"] == pytest.approx(2000.0)            # the reported value stays the cold one
+    assert cold["warm"]["us_per_call"] == pytest.approx(1500.0)
+    assert "not flushed" in cold["warm"]["l2"]
+    assert "warm" not in bench.result_line(sh, cm, _m(None), 1, 4, 3, PEAKS, "measured", False)
