@@ -65,3 +65,19 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch):
     monkeypatch.setattr(bench.W, "inputs", lambda *a, **k: called.append(1))
     assert bench.run_reference(bench.parse_args(["--impl", "reference", "--gpus", "2"])) == 0
     assert not called
+
+
+def test_reference_arm_line_on_rank0(monkeypatch, capsys):
+    import json
+
+    monkeypatch.setenv("RANK", "0")
+    args = bench.parse_args(["--impl", "reference", "--workload", "C1", "--tokens", "8", "--steps", "2",
+                             "--warmup", "1", "--cpu-threads", "2"])
+    assert bench.run_reference(args) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "TFLOP/s" and line["value"] > 0
+    assert line["steps"] == 2 and line["warmup"] == 1 and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 2
+    assert line["cpu_baseline"]["value"] == line["value"] == line["e2e"]["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert "C1" in line["config"]["workload"]
