@@ -213,3 +213,48 @@ def test_unrounded_dense_top1_matches_torch():
         a_bits = np.array([oracle.double_to_bf16(v) for v in a.numpy().ravel()], np.uint16).reshape(a.shape)
         ref = F.linear(torch.from_numpy(W.bf16_bits_to_f32(a_bits)).double(), _bf16_to_t(w2[e])).numpy()
         np.testing.assert_allclose(f64[rows], ref, rtol=1e-9, atol=1e-12)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "mxfp8"])
+def test_final_rounding_is_one_rounding_of_the_exact_sum(dtype):
+    """out = RNE_bf16 of the exact route sum, rounded once.
+
+    The inputs make the intermediate exactly 1:
+    - x = 8 in column 0;
+    - the gate row is 8, so g = 64 and silu(64) = 64 to double precision;
+    - the up row is 2^-9, so u = 1/64.
+    With w2 = +-1, each route's result is +-1. The token's two routes carry weights 1 + 2^-8 and 2^-30,
+    so the exact sum is 1 + 2^-8 + 2^-30. That lies just above the midpoint of the bf16 neighbours 1 and
+    1 + 2^-7, so it rounds up to 0x3F81. Rounding through fp32 first would land on the midpoint itself
+    and tie to even (0x3F80)."""
+    K, E = 32, 1
+    N = 4 if dtype == "bf16" else 64          # the mxfp8 path needs N/2 to be a multiple of 32
+    I = N // 2
+    ids = np.zeros((1, 2), np.int32)          # both routes to expert 0
+    tw = np.array([[1.0 + 2.0 ** -8, 2.0 ** -30]], np.float32)
+    assert float(tw[0, 0]) + float(tw[0, 1]) == 1.0 + 2.0 ** -8 + 2.0 ** -30
+    if dtype == "bf16":
+        bf = {8.0: 0x4100, 2.0 ** -9: 0x3B00, 1.0: 0x3F80, -1.0: 0xBF80}
+        x = np.zeros((1, K), np.uint16)
+        x[0, 0] = bf[8.0]
+        w1 = np.zeros((E, N, K), np.uint16)
+        w1[0, 0, 0], w1[0, I, 0] = bf[8.0], bf[2.0 ** -9]
+        w2 = np.zeros((E, K, I), np.uint16)
+        w2[0, 0, 0], w2[0, 1, 0] = bf[1.0], bf[-1.0]
+        out, f64 = oracle.fused_moe_bf16(x, w1, w2, ids, tw, unrounded=True)
+    else:
+        # e4m3 codes: 8.0 = 0x50, 1.0 = 0x38, -1.0 = 0xB8; e8m0 byte 127 = 2^0, 118 = 2^-9
+        x = np.zeros((1, K), np.uint8)
+        x[0, 0] = 0x50
+        xs = np.full((1, K // 32), 127, np.uint8)
+        w1 = np.zeros((E, N, K), np.uint8)
+        w1[0, 0, 0], w1[0, I, 0] = 0x50, 0x38
+        s1 = np.full((E, N, K // 32), 127, np.uint8)
+        s1[0, I, 0] = 118
+        w2 = np.zeros((E, K, I), np.uint8)
+        w2[0, 0, 0], w2[0, 1, 0] = 0x38, 0xB8
+        s2 = np.full((E, K, I // 32), 127, np.uint8)
+        out, f64 = oracle.fused_moe_mxfp8(x, xs, w1, s1, w2, s2, ids, tw, unrounded=True)
+    assert f64[0, 0] == 1.0 + 2.0 ** -8 + 2.0 ** -30 and f64[0, 1] == -f64[0, 0]
+    assert int(out[0, 0]) == 0x3F81 and int(out[0, 1]) == 0xBF81
+    assert not f64[0, 2:].any() and not out[0, 2:].any()
