@@ -22,7 +22,8 @@ def _has_gpu() -> bool:
 
 
 def pytest_collection_modifyitems(config, items):
-    if _has_gpu():
+    # torch is imported only when a GPU test was collected (a CPU-only selection stays light)
+    if not any("gpu" in item.keywords for item in items) or _has_gpu():
         return
     skip = pytest.mark.skip(reason="no CUDA device")
     for item in items:
