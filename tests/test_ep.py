@@ -1,4 +1,4 @@
-"""Expert-parallel forward (ep_forward) on two gloo ranks on CPU.
+"""Expert-parallel forward (ep_forward) on two and four gloo ranks on CPU.
 
 Each rank holds its own batch; the experts are split over the ranks.  The local compute is the
 oracle (tests may run it) on the rows a rank receives, so what is checked is the dispatch and the
@@ -90,9 +90,8 @@ def _worker(rank, world, port, mode, results):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("mode", ["mixed", "empty_rank", "one_rank"])
-def test_ep_forward_matches_the_single_process_oracle(mode):
-    world = 2
+@pytest.mark.parametrize("mode,world", [("mixed", 2), ("empty_rank", 2), ("one_rank", 2), ("mixed", 4)])
+def test_ep_forward_matches_the_single_process_oracle(mode, world):
     ctx = mp.get_context("spawn")
     with ctx.Manager() as mgr:
         results = mgr.dict()
@@ -104,7 +103,7 @@ def test_ep_forward_matches_the_single_process_oracle(mode):
             p.join(180)
             assert p.exitcode == 0
         res = dict(results)
-    assert res == {0: 0.0, 1: 0.0}, res
+    assert res == {r: 0.0 for r in range(world)}, res
 
 
 def test_owner_of():
