@@ -111,9 +111,14 @@ def cost_model(sh: W.Shape, topk_ids: np.ndarray, peaks: dict):
     bx = 2.0 if sh.dtype == "bf16" else 1.0 + 1.0 / 32.0
     p1_bytes = touched * sh.N * sh.K * b + R * sh.K * bx + R * sh.I * bx
     p1_flops = 2.0 * R * sh.K * sh.N
+    # the whole path's algorithmic HBM bytes: touched weights, x (+ its scales) read once, out written
+    # once, the routing read, the planner's arrays written (sorted ids, expert ids, the padded total)
+    cap = R + sh.E * (sh.block_m - 1)
+    full = {"weights": bytes_w, "x": sh.T * sh.K * bx, "out": 2.0 * sh.T * sh.K, "routing": 8.0 * R,
+            "plan": 4.0 * cap + 4.0 * ((cap + sh.block_m - 1) // sh.block_m) + 4.0}
     return dict(R=R, flops=flops, touched=touched, bytes_w=bytes_w, t_flop=t_flop, t_hbm=t_hbm,
                 t_roof=max(t_flop, t_hbm), bound="tensor" if t_flop > t_hbm else "hbm", p_tc=p_tc, bw=bw,
-                p1_bytes=p1_bytes, p1_flops=p1_flops)
+                p1_bytes=p1_bytes, p1_flops=p1_flops, bytes_full=sum(full.values()), bytes_parts=full)
 
 
 class ClockSampler:
@@ -499,6 +504,8 @@ def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
         "path_roofline": {"bound": cm["bound"], "t_roof_us": cm["t_roof"] * 1e6,
                           "frac": cm["t_roof"] / (ms_step * 1e-3), "touched_experts": cm["touched"],
                           "routed_gflop": cm["flops"] / 1e9, "touched_weight_gb": cm["bytes_w"] / 1e9,
+                          "algorithmic_hbm_gb": cm["bytes_full"] / 1e9,
+                          "algorithmic_hbm_parts_gb": {k: v / 1e9 for k, v in cm["bytes_parts"].items()},
                           "peaks": peak_src},
         "phase_us": {"planner": m["plan_ms"] * 1e3, "gate_up": m["p1_ms"] * 1e3, "down": m["p2_ms"] * 1e3,
                      "reduce": m["cb_ms"] * 1e3},

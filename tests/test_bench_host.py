@@ -57,3 +57,15 @@ def test_warm_time_is_reported_beside_the_cold_one():
     assert cold["warm"]["us_per_call"] == pytest.approx(1500.0)
     assert "not flushed" in cold["warm"]["l2"]
     assert "warm" not in bench.result_line(sh, cm, _m(None), 1, 4, 3, PEAKS, "measured", False)
+
+
+def test_full_algorithmic_bytes():
+    sh = W.shape("C2", 64)                                 # bf16, block_m 128
+    ids = np.tile(np.arange(sh.top_k, dtype=np.int32), (sh.T, 1))
+    cm = bench.cost_model(sh, ids, PEAKS)
+    R = sh.T * sh.top_k
+    cap = R + sh.E * (sh.block_m - 1)
+    want = (cm["bytes_w"] + 2 * sh.T * sh.K + 2 * sh.T * sh.K + 8 * R + 4 * cap
+            + 4 * ((cap + sh.block_m - 1) // sh.block_m) + 4)
+    assert cm["bytes_full"] == pytest.approx(want)
+    assert cm["bytes_full"] > cm["bytes_w"]
