@@ -397,9 +397,15 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
                 flush()
         t1.record(stream)
         torch.cuda.synchronize()
-        return sum(a.elapsed_time(b) for a, b in s_ev) if s_ev else t0.elapsed_time(t1)
+        if s_ev:
+            per_step.clear()
+            per_step.extend(a.elapsed_time(b) for a, b in s_ev)
+            return sum(per_step)
+        return t0.elapsed_time(t1)
 
+    per_step = []
     total_ms = timed()
+    median_ms = float(np.median(per_step)) if per_step else None
     if barrier:
         barrier()
     clk = clocks.stop() if clocks else None
@@ -415,7 +421,7 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
         prob.step()  # the last flush left L2 cold; one untimed step warms it
         warm_ms = timed(cold=False) / steps
         moe.moe_device_status()
-    return {"total_ms": total_ms, "ms_step": total_ms / steps, "warm_ms_step": warm_ms,
+    return {"total_ms": total_ms, "ms_step": total_ms / steps, "warm_ms_step": warm_ms, "median_ms_step": median_ms,
             "plan_ms": sum(a.elapsed_time(e[0]) for a, e in zip(pev, ev)) / steps,
             "p1_ms": sum(e[0].elapsed_time(e[1]) for e in ev) / steps,
             "p2_ms": sum(e[1].elapsed_time(e[2]) for e in ev) / steps,
@@ -500,6 +506,7 @@ def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
                                f"E={sh.E} top_k={sh.top_k} T={sh.T} block_m={sh.block_m}",
                    "tokens_per_gpu": sh.T, "parallelism": f"replicas x{world}", "l2": l2},
         "us_per_call": ms_step * 1e3,
+        **({"us_per_call_median": m["median_ms_step"] * 1e3} if m.get("median_ms_step") else {}),
         "weight_GBps": cm["bytes_w"] / (ms_step * 1e-3) / 1e9,
         "path_roofline": {"bound": cm["bound"], "t_roof_us": cm["t_roof"] * 1e6,
                           "frac": cm["t_roof"] / (ms_step * 1e-3), "touched_experts": cm["touched"],
