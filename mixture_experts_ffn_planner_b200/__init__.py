@@ -151,6 +151,42 @@ def _need(t, name, dtypes, device=True):
         raise ValueError(f"{name} must be a CUDA tensor")
 
 
+def _ffn_shapes(fmt: str, x, w1, w2, topk_weights, out, sorted_token_ids, expert_ids, num_tokens_post_padded,
+                block_m: int, x_scales=None, w1_scales=None, w2_scales=None):
+    """The C ABI takes its sizes from x and w1 and trusts every other buffer, so the shapes (and the
+    device) of all of them are checked here before a launch: a short buffer would be read or written
+    out of bounds by the kernels.  fmt: "bf16", "mxfp8" or "mxfp4" (packed weights, two per byte)."""
+    if x.dim() != 2 or w1.dim() != 3:
+        raise ValueError("x must be (T, K) and w1 (E, N, K)")
+    T, K = x.shape
+    E, N = w1.shape[0], w1.shape[1]
+    pack = 2 if fmt == "mxfp4" else 1
+    if N % 2:
+        raise ValueError(f"N = {N} must be even (gate and up halves)")
+    want = {"w1": (E, N, K // pack), "w2": (E, K, N // 2 // pack), "out": (T, K)}
+    for name, t in (("w1", w1), ("w2", w2), ("out", out)):
+        if tuple(t.shape) != want[name]:
+            raise ValueError(f"{name} must have shape {want[name]}, got {tuple(t.shape)}")
+    if topk_weights.dim() != 2 or topk_weights.shape[0] != T:
+        raise ValueError(f"topk_weights must be (T={T}, top_k), got {tuple(topk_weights.shape)}")
+    if expert_ids.numel() < (sorted_token_ids.numel() + block_m - 1) // block_m or num_tokens_post_padded.numel() < 1:
+        raise ValueError("expert_ids must hold ceil(sorted_token_ids.numel() / block_m) entries and "
+                         "num_tokens_post_padded one")
+    tensors = [w1, w2, out, topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded]
+    if fmt != "bf16":
+        if tuple(x_scales.shape) != (T, K // 32):
+            raise ValueError(f"x_scales must have shape {(T, K // 32)}, got {tuple(x_scales.shape)}")
+        for name, t, mn, ks in (("w1_scales_blocked", w1_scales, N, K // 32),
+                                ("w2_scales_blocked", w2_scales, K, N // 2 // 32)):
+            need = pack_scales_blocked_bytes(E, mn, ks)
+            if t.numel() < need:
+                raise ValueError(f"{name} must hold {need} bytes (pack_scales_blocked of ({E}, {mn}, {ks}))")
+        tensors += [x_scales, w1_scales, w2_scales]
+    for t in tensors:
+        if t.device != x.device:
+            raise ValueError(f"all tensors must be on {x.device}, got one on {t.device}")
+
+
 # ---------------------------------------------------------------- sizes
 def moe_align_capacity(T: int, top_k: int, E: int, block_m: int) -> int:
     return int(load().moe_align_capacity(T, top_k, E, block_m))
@@ -278,6 +314,7 @@ def fused_moe_bf16(x, w1, w2, sorted_token_ids, expert_ids, num_tokens_post_padd
     for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
                  (num_tokens_post_padded, "num_tokens_post_padded")):
         _need(t, n, (torch.int32,))
+    _ffn_shapes("bf16", x, w1, w2, topk_weights, out, sorted_token_ids, expert_ids, num_tokens_post_padded, block_m)
     T, K = x.shape
     E, N, _ = w1.shape
     top_k = topk_weights.shape[1]
@@ -306,6 +343,8 @@ def fused_moe_mxfp8(x, x_scales, w1, w1_scales_blocked, w2, w2_scales_blocked, s
     for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
                  (num_tokens_post_padded, "num_tokens_post_padded")):
         _need(t, n, (torch.int32,))
+    _ffn_shapes("mxfp8", x, w1, w2, topk_weights, out, sorted_token_ids, expert_ids, num_tokens_post_padded, block_m,
+                x_scales, w1_scales_blocked, w2_scales_blocked)
     T, K = x.shape
     E, N, _ = w1.shape
     top_k = topk_weights.shape[1]
@@ -334,10 +373,10 @@ def fused_moe_mxfp4(x, x_scales, w1, w1_scales_blocked, w2, w2_scales_blocked, s
     for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
                  (num_tokens_post_padded, "num_tokens_post_padded")):
         _need(t, n, (torch.int32,))
+    _ffn_shapes("mxfp4", x, w1, w2, topk_weights, out, sorted_token_ids, expert_ids, num_tokens_post_padded, block_m,
+                x_scales, w1_scales_blocked, w2_scales_blocked)
     T, K = x.shape
-    E, N, Kh = w1.shape
-    if Kh * 2 != K:
-        raise ValueError("w1 must be (E, N, K/2) packed e2m1")
+    E, N, _ = w1.shape
     top_k = topk_weights.shape[1]
     ws = _workspace(DTYPE_MXFP4, T, K, N, E, top_k, block_m, workspace, x.device)
     _check(load().fused_moe_mxfp4(
@@ -367,6 +406,7 @@ def fused_moe_bf16_noalloc(x, w1, w2, sorted_token_ids, expert_ids, num_tokens_p
     for t, n in ((sorted_token_ids, "sorted_token_ids"), (expert_ids, "expert_ids"),
                  (num_tokens_post_padded, "num_tokens_post_padded")):
         _need(t, n, (torch.int32,))
+    _ffn_shapes("bf16", x, w1, w2, topk_weights, out, sorted_token_ids, expert_ids, num_tokens_post_padded, block_m)
     T, K = x.shape
     E, N, _ = w1.shape
     top_k = topk_weights.shape[1]
