@@ -32,12 +32,14 @@ def owner_of(expert_ids, E: int, world: int):
     return torch.where(valid, torch.div(expert_ids, per, rounding_mode="floor"), torch.full_like(expert_ids, -1))
 
 
-def ep_forward(x, topk_ids, topk_weights, E: int, local_ffn: Callable, group=None):
+def ep_forward(x, topk_ids, topk_weights, E: int, local_ffn: Callable, group=None, x_scales=None):
     """Expert-parallel MoE forward of this rank's tokens.
 
-    x (T, K) rows of this rank; topk_ids (T, k) int32 global expert ids (ids outside [0, E) route
-    nowhere); topk_weights (T, k) fp32.  local_ffn(rows (M, K), local_expert (M,) int32, weight (M,) fp32)
-    returns the weighted expert outputs (M, K) of the rows this rank received (any float dtype).
+    x (T, K) rows of this rank (bf16 values, or e4m3 codes as uint8); topk_ids (T, k) int32 global
+    expert ids (ids outside [0, E) route nowhere); topk_weights (T, k) fp32.  x_scales (T, K/32) uint8
+    e8m0, for e4m3 rows: each row's scales travel with it.  local_ffn(rows (M, K), local_expert (M,)
+    int32, weight (M,) fp32[, row_scales (M, K/32) when x_scales is given]) returns the weighted expert
+    outputs (M, K) of the rows this rank received (any float dtype).
     Returns out (T, K) in local_ffn's dtype: for every token the sum, in route order, of its routes'
     weighted expert outputs.  E must be a multiple of the group size.
     """
@@ -72,8 +74,13 @@ def ep_forward(x, topk_ids, topk_weights, E: int, local_ffn: Callable, group=Non
     dist.all_to_all_single(rows_in, rows_out, rc, sc, group=group)
     dist.all_to_all_single(local_e_in, local_e_out, rc, sc, group=group)
     dist.all_to_all_single(w_in, w_out, rc, sc, group=group)
-
-    y_in = local_ffn(rows_in, local_e_in, w_in)               # (M, K) weighted outputs of received routes
+    if x_scales is not None:
+        sc_out = x_scales[torch.div(order, k, rounding_mode="floor")].contiguous()
+        sc_in = torch.empty((M, x_scales.shape[1]), dtype=x_scales.dtype, device=dev)
+        dist.all_to_all_single(sc_in, sc_out, rc, sc, group=group)
+        y_in = local_ffn(rows_in, local_e_in, w_in, sc_in)
+    else:
+        y_in = local_ffn(rows_in, local_e_in, w_in)           # (M, K) weighted outputs of received routes
     y_back = torch.empty((len(order), K), dtype=y_in.dtype, device=dev)
     dist.all_to_all_single(y_back, y_in.contiguous(), sc, rc, group=group)
 

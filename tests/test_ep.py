@@ -4,7 +4,8 @@ Each rank holds its own batch; the experts are split over the ranks.  The local 
 oracle (tests may run it) on the rows a rank receives, so what is checked is the dispatch and the
 combine: every rank's result must equal the single-process oracle on that rank's tokens with all
 experts, in float64 to the last bit (routes are summed in the same order).  Covers routes that cross
-ranks, routes to nowhere (id -1), a rank with no tokens, and all routes landing on one rank.
+ranks, routes to nowhere (id -1), a rank with no tokens, and all routes landing on one rank; on the
+mxfp8 path each row's e8m0 scales travel with its e4m3 codes.
 The GPU ranks of this path (NCCL between B200s) are not exercised here: every GPU run here has one
 GPU.
 """
@@ -50,7 +51,13 @@ def _batch(rank, T, k, mode):
     return x, ids, w
 
 
-def _worker(rank, world, port, mode, results):
+def _mx(a):
+    import workloads as W
+
+    return W.mx_quantize_inputs(W.bf16_bits_to_f32(a))
+
+
+def _worker(rank, world, port, mode, results, fmt="bf16"):
     import datetime
 
     import torch.distributed as dist
@@ -67,21 +74,35 @@ def _worker(rank, world, port, mode, results):
         lo = rank * per
         T = 0 if (mode == "empty_rank" and rank == 0) else 9 + 4 * rank
         x, ids, tw = _batch(rank, T, 2, mode)
+        if fmt == "mxfp8":
+            (w1q, w1s), (w2q, w2s) = _mx(w1), _mx(w2)
+            xq, xs = _mx(x) if T else (np.zeros((0, K), np.uint8), np.zeros((0, K // 32), np.uint8))
 
-        def local_ffn(rows, local_e, weight):
+        def local_ffn(rows, local_e, weight, row_scales=None):
             M = rows.shape[0]
             if M == 0:
                 return torch.zeros((0, K), dtype=torch.float64)
-            bits = W.f32_to_bf16_bits(rows.numpy().astype(np.float32))   # exact: rows hold bf16 values
-            y = oracle.fused_moe_bf16(bits, w1[lo:lo + per], w2[lo:lo + per],
-                                      local_e.numpy().reshape(M, 1).astype(np.int32),
-                                      weight.numpy().reshape(M, 1).astype(np.float32), unrounded=True)[1]
+            le = local_e.numpy().reshape(M, 1).astype(np.int32)
+            wt = weight.numpy().reshape(M, 1).astype(np.float32)
+            if fmt == "mxfp8":
+                y = oracle.fused_moe_mxfp8(rows.numpy(), row_scales.numpy(), w1q[lo:lo + per], w1s[lo:lo + per],
+                                           w2q[lo:lo + per], w2s[lo:lo + per], le, wt, unrounded=True)[1]
+            else:
+                bits = W.f32_to_bf16_bits(rows.numpy().astype(np.float32))   # exact: rows hold bf16 values
+                y = oracle.fused_moe_bf16(bits, w1[lo:lo + per], w2[lo:lo + per], le, wt, unrounded=True)[1]
             return torch.from_numpy(y)
 
-        xt = torch.from_numpy(W.bf16_bits_to_f32(x)) if T else torch.zeros((0, K), dtype=torch.float32)
-        out = ep_forward(xt, torch.from_numpy(ids).reshape(T, 2), torch.from_numpy(tw).reshape(T, 2), E, local_ffn)
+        ids_t, tw_t = torch.from_numpy(ids).reshape(T, 2), torch.from_numpy(tw).reshape(T, 2)
+        if fmt == "mxfp8":
+            out = ep_forward(torch.from_numpy(xq), ids_t, tw_t, E, local_ffn, x_scales=torch.from_numpy(xs))
+        else:
+            xt = torch.from_numpy(W.bf16_bits_to_f32(x)) if T else torch.zeros((0, K), dtype=torch.float32)
+            out = ep_forward(xt, ids_t, tw_t, E, local_ffn)
         if T:
-            ref = oracle.fused_moe_bf16(x, w1, w2, ids, tw, unrounded=True)[1]
+            if fmt == "mxfp8":
+                ref = oracle.fused_moe_mxfp8(xq, xs, w1q, w1s, w2q, w2s, ids, tw, unrounded=True)[1]
+            else:
+                ref = oracle.fused_moe_bf16(x, w1, w2, ids, tw, unrounded=True)[1]
             results[rank] = float(np.max(np.abs(out.numpy() - ref)))
         else:
             results[rank] = 0.0 if out.shape == (0, K) else -1.0
@@ -90,13 +111,14 @@ def _worker(rank, world, port, mode, results):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("mode,world", [("mixed", 2), ("empty_rank", 2), ("one_rank", 2), ("mixed", 4)])
-def test_ep_forward_matches_the_single_process_oracle(mode, world):
+@pytest.mark.parametrize("mode,world,fmt", [("mixed", 2, "bf16"), ("empty_rank", 2, "bf16"), ("one_rank", 2, "bf16"),
+                                             ("mixed", 4, "bf16"), ("mixed", 2, "mxfp8"), ("empty_rank", 2, "mxfp8")])
+def test_ep_forward_matches_the_single_process_oracle(mode, world, fmt):
     ctx = mp.get_context("spawn")
     with ctx.Manager() as mgr:
         results = mgr.dict()
         port = _free_port()
-        procs = [ctx.Process(target=_worker, args=(r, world, port, mode, results)) for r in range(world)]
+        procs = [ctx.Process(target=_worker, args=(r, world, port, mode, results, fmt)) for r in range(world)]
         for p in procs:
             p.start()
         for p in procs:
