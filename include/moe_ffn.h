@@ -151,7 +151,9 @@ MOE_API int pack_scales_blocked(const uint8_t* in, uint8_t* out, int E, int MN, 
                         moe_stream_t stream);
 
 /* ------------------------------------------------------------------------
- * Workspace.  fused_moe_* need caller-owned device scratch of at least
+ * Workspace -- [PFM] intro, the split=True form: the activation is written
+ * to a workspace once and read back by the down projection.
+ * fused_moe_* need caller-owned device scratch of at least
  * moe_workspace_bytes(...) bytes, 256-byte aligned.  It holds the SwiGLU
  * intermediate of every routed row (written once, read once by the down
  * projection), the weighted down-projection rows of every route, and one

@@ -25,6 +25,7 @@ Entry points (same names as the C ABI):
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -132,12 +133,32 @@ def _ptr(t) -> int | None:
     return None if t is None else t.data_ptr()
 
 
-def _stream(stream) -> int | None:
+@contextlib.contextmanager
+def _on_device(dev, stream):
+    """Makes ``dev`` (the device of the call's tensors) the current CUDA device
+    for the C call and yields the stream handle to launch on.
+
+    The library launches on the current device and builds its TMA descriptors
+    from the tensors' addresses, so a call whose tensors live on another
+    device than the current one would read that device's memory from the
+    wrong GPU.  ``stream``: None (the current stream of ``dev``), a
+    ``torch.cuda.Stream`` (must belong to ``dev``) or a raw ``cudaStream_t``
+    handle as an int (the caller vouches for its device)."""
     import torch
 
-    if stream is None:
-        stream = torch.cuda.current_stream()
-    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    if getattr(dev, "type", None) != "cuda":
+        raise ValueError(f"tensors must be on a CUDA device, got {dev}")
+    with torch.cuda.device(dev):
+        if stream is None:
+            handle = torch.cuda.current_stream(dev).cuda_stream
+        elif hasattr(stream, "cuda_stream"):
+            sdev = getattr(stream, "device", dev)
+            if torch.device(sdev) != torch.device(dev):
+                raise ValueError(f"stream belongs to {sdev} but the tensors are on {dev}")
+            handle = stream.cuda_stream
+        else:
+            handle = int(stream)
+        yield handle
 
 
 def _need(t, name, dtypes, device=True):
@@ -187,6 +208,12 @@ def _ffn_shapes(fmt: str, x, w1, w2, topk_weights, out, sorted_token_ids, expert
             raise ValueError(f"all tensors must be on {x.device}, got one on {t.device}")
 
 
+def _same_device(first, *rest):
+    for t in rest:
+        if t.device != first.device:
+            raise ValueError(f"all tensors must be on {first.device}, got one on {t.device}")
+
+
 # ---------------------------------------------------------------- sizes
 def moe_align_capacity(T: int, top_k: int, E: int, block_m: int) -> int:
     return int(load().moe_align_capacity(T, top_k, E, block_m))
@@ -227,8 +254,10 @@ def moe_align(topk_ids, E: int, block_m: int, sorted_token_ids=None, expert_ids=
         _need(t, n, (torch.int32,))
     if expert_ids.numel() < (sorted_token_ids.numel() + block_m - 1) // block_m:
         raise ValueError("expert_ids must hold ceil(capacity / block_m) entries")
-    _check(load().moe_align(_ptr(topk_ids), T, top_k, E, block_m, _ptr(sorted_token_ids), _ptr(expert_ids),
-                            _ptr(num_tokens_post_padded), sorted_token_ids.numel(), _stream(stream)))
+    _same_device(topk_ids, sorted_token_ids, expert_ids, num_tokens_post_padded)
+    with _on_device(topk_ids.device, stream) as s:
+        _check(load().moe_align(_ptr(topk_ids), T, top_k, E, block_m, _ptr(sorted_token_ids), _ptr(expert_ids),
+                                _ptr(num_tokens_post_padded), sorted_token_ids.numel(), s))
     return sorted_token_ids, expert_ids, num_tokens_post_padded
 
 
@@ -271,9 +300,12 @@ def moe_route_align(logits, top_k: int, block_m: int, bias=None, topk_ids=None, 
         _need(t, n, (torch.int32,))
     if expert_ids.numel() < (sorted_token_ids.numel() + block_m - 1) // block_m:
         raise ValueError("expert_ids must hold ceil(capacity / block_m) entries")
-    _check(load().moe_route_align(_ptr(logits), _ptr(bias), T, E, top_k, n_shared, block_m, _ptr(topk_ids),
-                                  _ptr(topk_weights), _ptr(sorted_token_ids), _ptr(expert_ids),
-                                  _ptr(num_tokens_post_padded), sorted_token_ids.numel(), _stream(stream)))
+    _same_device(logits, *([] if bias is None else [bias]), topk_ids, topk_weights, sorted_token_ids, expert_ids,
+                 num_tokens_post_padded)
+    with _on_device(logits.device, stream) as s:
+        _check(load().moe_route_align(_ptr(logits), _ptr(bias), T, E, top_k, n_shared, block_m, _ptr(topk_ids),
+                                      _ptr(topk_weights), _ptr(sorted_token_ids), _ptr(expert_ids),
+                                      _ptr(num_tokens_post_padded), sorted_token_ids.numel(), s))
     return topk_ids, topk_weights, sorted_token_ids, expert_ids, num_tokens_post_padded
 
 
@@ -289,7 +321,9 @@ def pack_scales_blocked(scales, out=None, stream=None):
     _need(out, "out", (torch.uint8,))
     if out.numel() < n:
         raise ValueError(f"out must hold {n} bytes")
-    _check(load().pack_scales_blocked(_ptr(scales), _ptr(out), E, MN, KS, _stream(stream)))
+    _same_device(scales, out)
+    with _on_device(scales.device, stream) as s:
+        _check(load().pack_scales_blocked(_ptr(scales), _ptr(out), E, MN, KS, s))
     return out
 
 
@@ -319,10 +353,12 @@ def fused_moe_bf16(x, w1, w2, sorted_token_ids, expert_ids, num_tokens_post_padd
     E, N, _ = w1.shape
     top_k = topk_weights.shape[1]
     ws = _workspace(DTYPE_BF16, T, K, N, E, top_k, block_m, workspace, x.device)
-    _check(load().fused_moe_bf16(
-        _ptr(x), _ptr(w1), _ptr(w2), _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded),
-        _ptr(topk_weights), _ptr(out), T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws), ws.numel(),
-        None if tune is None else ctypes.byref(tune), _stream(stream)))
+    _same_device(x, ws)
+    with _on_device(x.device, stream) as s:
+        _check(load().fused_moe_bf16(
+            _ptr(x), _ptr(w1), _ptr(w2), _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded),
+            _ptr(topk_weights), _ptr(out), T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws),
+            ws.numel(), None if tune is None else ctypes.byref(tune), s))
     return out
 
 
@@ -349,11 +385,13 @@ def fused_moe_mxfp8(x, x_scales, w1, w1_scales_blocked, w2, w2_scales_blocked, s
     E, N, _ = w1.shape
     top_k = topk_weights.shape[1]
     ws = _workspace(DTYPE_MXFP8, T, K, N, E, top_k, block_m, workspace, x.device)
-    _check(load().fused_moe_mxfp8(
-        _ptr(x), _ptr(x_scales), _ptr(w1), _ptr(w1_scales_blocked), _ptr(w2), _ptr(w2_scales_blocked),
-        _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(topk_weights), _ptr(out),
-        T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws), ws.numel(),
-        None if tune is None else ctypes.byref(tune), _stream(stream)))
+    _same_device(x, ws)
+    with _on_device(x.device, stream) as s:
+        _check(load().fused_moe_mxfp8(
+            _ptr(x), _ptr(x_scales), _ptr(w1), _ptr(w1_scales_blocked), _ptr(w2), _ptr(w2_scales_blocked),
+            _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(topk_weights), _ptr(out),
+            T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws), ws.numel(),
+            None if tune is None else ctypes.byref(tune), s))
     return out
 
 
@@ -379,11 +417,13 @@ def fused_moe_mxfp4(x, x_scales, w1, w1_scales_blocked, w2, w2_scales_blocked, s
     E, N, _ = w1.shape
     top_k = topk_weights.shape[1]
     ws = _workspace(DTYPE_MXFP4, T, K, N, E, top_k, block_m, workspace, x.device)
-    _check(load().fused_moe_mxfp4(
-        _ptr(x), _ptr(x_scales), _ptr(w1), _ptr(w1_scales_blocked), _ptr(w2), _ptr(w2_scales_blocked),
-        _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(topk_weights), _ptr(out),
-        T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws), ws.numel(),
-        None if tune is None else ctypes.byref(tune), _stream(stream)))
+    _same_device(x, ws)
+    with _on_device(x.device, stream) as s:
+        _check(load().fused_moe_mxfp4(
+            _ptr(x), _ptr(x_scales), _ptr(w1), _ptr(w1_scales_blocked), _ptr(w2), _ptr(w2_scales_blocked),
+            _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded), _ptr(topk_weights), _ptr(out),
+            T, K, N, E, top_k, block_m, sorted_token_ids.numel(), _ptr(ws), ws.numel(),
+            None if tune is None else ctypes.byref(tune), s))
     return out
 
 
@@ -410,13 +450,20 @@ def fused_moe_bf16_noalloc(x, w1, w2, sorted_token_ids, expert_ids, num_tokens_p
     T, K = x.shape
     E, N, _ = w1.shape
     top_k = topk_weights.shape[1]
-    _check(load().fused_moe_bf16_noalloc(
-        _ptr(x), _ptr(w1), _ptr(w2), _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded),
-        _ptr(topk_weights), _ptr(out), T, K, N, E, top_k, block_m, sorted_token_ids.numel(),
-        None if tune is None else ctypes.byref(tune), _stream(stream)))
+    with _on_device(x.device, stream) as s:
+        _check(load().fused_moe_bf16_noalloc(
+            _ptr(x), _ptr(w1), _ptr(w2), _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded),
+            _ptr(topk_weights), _ptr(out), T, K, N, E, top_k, block_m, sorted_token_ids.numel(),
+            None if tune is None else ctypes.byref(tune), s))
     return out
 
 
-def moe_device_status(stream=None):
-    """Waits for the stream; raises MoeError(MOE_ERR_TIMEOUT) if a device-side wait gave up."""
-    _check(load().moe_device_status(_stream(stream)))
+def moe_device_status(stream=None, device=None):
+    """Waits for the stream; raises MoeError(MOE_ERR_TIMEOUT) if a device-side wait of this library
+    on that device gave up.  ``device``: default the stream's device, else the current one."""
+    import torch
+
+    if device is None:
+        device = getattr(stream, "device", None) or torch.device("cuda", torch.cuda.current_device())
+    with _on_device(torch.device(device), stream) as s:
+        _check(load().moe_device_status(s))

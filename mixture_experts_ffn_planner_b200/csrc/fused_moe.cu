@@ -1235,7 +1235,11 @@ static int pick_stages(int stage_bytes, int ctrl, int requested, int max_stages)
   return s;
 }
 
-static int run_fused(const FusedArgs& a) {
+// Every argument check of the fused forward that does not depend on the
+// workspace, in the order the status codes are documented.  Returns MOE_OK or
+// the error status (message in moe_last_error()).  `has_ws`: the workspace
+// pointer is checked for null and alignment as well.
+static int check_fused(const FusedArgs& a, bool has_ws) {
   const char* nm = a.w_fp4 ? "fused_moe_mxfp4" : (a.fp8 ? "fused_moe_mxfp8" : "fused_moe_bf16");
   if (a.T < 0 || a.K <= 0 || a.N <= 0 || a.E < 1 || a.top_k < 1)
     return fail(MOE_ERR_INVALID_ARG, "%s: need T >= 0, K > 0, N > 0, E >= 1, top_k >= 1", nm);
@@ -1255,15 +1259,24 @@ static int run_fused(const FusedArgs& a) {
   if (static_cast<int64_t>(a.E) * a.N >= (int64_t(1) << 31) || static_cast<int64_t>(a.E) * a.K >= (int64_t(1) << 31))
     return fail(MOE_ERR_UNSUPPORTED, "%s: E*N and E*K must be < 2^31", nm);
   if (a.T == 0) return MOE_OK;
-  if (!a.x || !a.w1 || !a.w2 || !a.sorted_ids || !a.expert_ids || !a.ntpp || !a.topk_w || !a.out || !a.ws)
+  if (!a.x || !a.w1 || !a.w2 || !a.sorted_ids || !a.expert_ids || !a.ntpp || !a.topk_w || !a.out ||
+      (has_ws && !a.ws))
     return fail(MOE_ERR_INVALID_ARG, "%s: null pointer", nm);
   if (a.fp8 && (!a.x_sf || !a.w1_sf || !a.w2_sf)) return fail(MOE_ERR_INVALID_ARG, "%s: null scale pointer", nm);
   if (!aligned(a.x, 16) || !aligned(a.w1, 16) || !aligned(a.w2, 16) || !aligned(a.out, 16) ||
-      !aligned(a.ws, 256) || (a.fp8 && (!aligned(a.x_sf, 16) || !aligned(a.w1_sf, 16) || !aligned(a.w2_sf, 16))) ||
+      (has_ws && !aligned(a.ws, 256)) ||
+      (a.fp8 && (!aligned(a.x_sf, 16) || !aligned(a.w1_sf, 16) || !aligned(a.w2_sf, 16))) ||
       !aligned(a.sorted_ids, 4) || !aligned(a.expert_ids, 4) || !aligned(a.ntpp, 4) || !aligned(a.topk_w, 4))
     return fail(MOE_ERR_ALIGNMENT, "%s: tensors must be 16-byte aligned and the workspace 256-byte aligned", nm);
   if (a.w_fp4 && (!aligned(a.w1, 32) || !aligned(a.w2, 32)))
     return fail(MOE_ERR_ALIGNMENT, "%s: packed e2m1 weights must be 32-byte aligned", nm);
+  return MOE_OK;
+}
+
+static int run_fused(const FusedArgs& a) {
+  const char* nm = a.w_fp4 ? "fused_moe_mxfp4" : (a.fp8 ? "fused_moe_mxfp8" : "fused_moe_bf16");
+  int rc0 = check_fused(a, true);
+  if (rc0 != MOE_OK || a.T == 0) return rc0;
   const WsLayout L = ws_layout(a.fp8, a.T, a.K, a.N, a.E, a.top_k, a.bm);
   if (a.ws_bytes < L.total)
     return fail(MOE_ERR_WORKSPACE, "%s: workspace %lld bytes < required %lld", nm, (long long)a.ws_bytes,
@@ -1558,9 +1571,16 @@ extern "C" int fused_moe_bf16_noalloc(const void* x, const void* w1, const void*
                                       const int32_t* num_tokens_post_padded, const float* topk_weights, void* out,
                                       int T, int K, int N, int E, int top_k, int block_m, int64_t capacity,
                                       const moe_tuning* tune, moe_stream_t stream) {
+  // The same argument checks, and so the same status codes, as fused_moe_bf16;
+  // only then the size limit of the built-in scratch.
+  moe::FusedArgs a{};
+  a.x = x; a.w1 = w1; a.w2 = w2;
+  a.sorted_ids = sorted_token_ids; a.expert_ids = expert_ids; a.ntpp = num_tokens_post_padded;
+  a.topk_w = topk_weights; a.out = out;
+  a.T = T; a.K = K; a.N = N; a.E = E; a.top_k = top_k; a.bm = block_m; a.capacity = capacity;
+  const int rc0 = moe::check_fused(a, false);
+  if (rc0 != MOE_OK || T == 0) return rc0;
   const int64_t need = moe_workspace_bytes(MOE_DTYPE_BF16, T, K, N, E, top_k, block_m);
-  if (need < 0)
-    return moe::fail(MOE_ERR_INVALID_ARG, "fused_moe_bf16_noalloc: invalid sizes");
   if (need > moe::kNoAllocScratchBytes)
     return moe::fail(MOE_ERR_WORKSPACE,
                      "fused_moe_bf16_noalloc: this problem needs %lld bytes of workspace, more than the %lld-byte "

@@ -141,3 +141,18 @@ def test_fused_rejects(lib):
     assert _mx(lib, ws=4096) == WORKSPACE
     msg = lib.moe_last_error()
     assert isinstance(msg, bytes) and b"workspace" in msg
+
+
+def _noalloc(lib, T=64, K=1024, N=1024, E=8, k=2, bm=64, cap=None, p=256):
+    cap = lib.moe_align_capacity(T, k, E, bm) if cap is None else cap
+    return lib.fused_moe_bf16_noalloc(p, p, p, p, p, p, p, p, T, K, N, E, k, bm, cap, None, None)
+
+
+def test_noalloc_rejects_like_fused_bf16(lib):
+    """Bad sizes give the no-allocation call the same status as fused_moe_bf16."""
+    for kw, code in ((dict(bm=48), UNSUPPORTED), (dict(T=-1), INVALID), (dict(E=0), INVALID),
+                     (dict(k=0), INVALID), (dict(K=1000), UNSUPPORTED), (dict(N=1000), UNSUPPORTED),
+                     (dict(cap=10), INVALID), (dict(p=0), INVALID), (dict(p=258), ALIGNMENT)):
+        assert _noalloc(lib, **kw) == code, kw
+        assert _bf16(lib, **kw) == code, kw
+    assert _noalloc(lib, T=0) == OK
