@@ -79,6 +79,8 @@ def _load():
         lib.orc_fused_moe_mxfp8.restype = None
         lib.orc_fused_moe_mxfp4.argtypes = lib.orc_fused_moe_mxfp8.argtypes
         lib.orc_fused_moe_mxfp4.restype = None
+        lib.orc_mx_intermediate.argtypes = [P, P, P, P, P, I, I, I, I, I, P, I, P, I, I]
+        lib.orc_mx_intermediate.restype = None
         lib.orc_e2m1_to_double.argtypes = [ctypes.c_uint8]
         lib.orc_e2m1_to_double.restype = ctypes.c_double
         lib.orc_max_threads.argtypes = []
@@ -259,6 +261,27 @@ def fused_moe_mxfp4(x, x_scales, w1, w1_scales, w2, w2_scales, topk_ids, topk_we
                                 _ptr(tw), T, K, N, E, top_k, None if t is None else _ptr(t), n,
                                 _ptr(out), None if f64 is None else _ptr(f64), int(nthreads))
     return (out, f64) if unrounded else out
+
+
+def mx_intermediate(x, x_scales, w1, w1_scales, topk_ids, tokens=None, nthreads: int = 0, fp4: bool = False,
+                    out=None):
+    """The fp32 SwiGLU intermediate of the mxfp8 forward (MXFP4 weights with ``fp4``) before its
+    requant: float32 (n, top_k, N/2) for the n listed tokens (all T when ``tokens`` is None), routes in
+    top-k order; a route to an expert outside [0, E) gives a zero row.  Scales row-major as for
+    fused_moe_mxfp8; w1 (E, N, K) e4m3 codes, or (E, N, K/2) packed e2m1 codes with ``fp4``."""
+    arrs = [np.ascontiguousarray(a, dtype=np.uint8) for a in (x, x_scales, w1, w1_scales)]
+    x, xs, w1, s1 = arrs
+    ids = np.ascontiguousarray(topk_ids, dtype=np.int32)
+    T, K = x.shape
+    E, N, Kw = w1.shape
+    assert Kw * (2 if fp4 else 1) == K and xs.shape == (T, K // 32) and s1.shape == (E, N, K // 32)
+    top_k = ids.shape[1]
+    t, n = _tokens_arg(tokens, T)
+    act = np.empty((n, top_k, N // 2), dtype=np.float32) if out is None else out
+    assert act.shape == (n, top_k, N // 2) and act.dtype == np.float32 and act.flags["C_CONTIGUOUS"]
+    _load().orc_mx_intermediate(_ptr(x), _ptr(xs), _ptr(w1), _ptr(s1), _ptr(ids), T, K, N, E, top_k,
+                                None if t is None else _ptr(t), n, _ptr(act), int(nthreads), int(bool(fp4)))
+    return act
 
 
 def e2m1_to_double(code: int) -> float:

@@ -389,10 +389,46 @@ void orc_fused_moe_bf16(const uint16_t* x, const uint16_t* w1, const uint16_t* w
  * code value: e4m3 (one byte per value) or e2m1 (two values per byte, the
  * even-indexed value in the low nibble -- reading: the usual packing order,
  * which the pages do not state). */
-static double weight_code(const uint8_t* W, int64_t idx, int fp4) {
-  if (!fp4) return orc_e4m3_to_double(W[idx]);
+/* Decoded values of every code, filled from the decoders above (a lookup
+ * of the same exact values, so that the sums below do not call ldexp per
+ * element; results are bit for bit those of calling the decoders). */
+typedef struct {
+  double e4m3[256], e8m0[256], e2m1[16];
+} decode_tables;
+
+static void fill_decode_tables(decode_tables* d) {
+  for (int c = 0; c < 256; ++c) {
+    d->e4m3[c] = orc_e4m3_to_double((uint8_t)c);
+    d->e8m0[c] = orc_e8m0_to_double((uint8_t)c);
+  }
+  for (int c = 0; c < 16; ++c) d->e2m1[c] = orc_e2m1_to_double((uint8_t)c);
+}
+
+static double weight_code(const decode_tables* d, const uint8_t* W, int64_t idx, int fp4) {
+  if (!fp4) return d->e4m3[W[idx]];
   const uint8_t b = W[idx >> 1];
-  return orc_e2m1_to_double((idx & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 0xF));
+  return d->e2m1[(idx & 1) ? (b >> 4) : (b & 0xF)];
+}
+
+/* One routed row's SwiGLU intermediate before the requant: H = w1[e] x
+ * (dequantised operands, double sums), af_i = fp32( silu(H_i) * H_{I+i} ).
+ * xd holds x[t] dequantised; H is scratch of N doubles. */
+static void mx_route_intermediate(const decode_tables* d, const double* xd, const uint8_t* W1, const uint8_t* S1,
+                                  int K, int N, int fp4, double* H, float* af) {
+  const int I = N / 2, KS = K / 32;
+  for (int n = 0; n < N; ++n) {
+    double s = 0.0;
+    for (int k = 0; k < K; ++k)
+      s += weight_code(d, W1, (int64_t)n * K + k, fp4) * d->e8m0[S1[(int64_t)n * KS + k / 32]] * xd[k];
+    H[n] = s;
+  }
+  for (int i = 0; i < I; ++i) af[i] = (float)(silu(H[i]) * H[I + i]);
+}
+
+/* x[t] dequantised exactly: e4m3 value times its e8m0 block scale (per 32 along K). */
+static void dequant_x(const decode_tables* d, const uint8_t* x, const uint8_t* x_scales, int t, int K, double* xd) {
+  const int KS = K / 32;
+  for (int k = 0; k < K; ++k) xd[k] = d->e4m3[x[(int64_t)t * K + k]] * d->e8m0[x_scales[(int64_t)t * KS + k / 32]];
 }
 
 static void fused_moe_mx(const uint8_t* x, const uint8_t* x_scales,
@@ -405,6 +441,9 @@ static void fused_moe_mx(const uint8_t* x, const uint8_t* x_scales,
   const int I = N / 2;
   const int KS = K / 32, IS = I / 32;
   const int count = tokens ? n_tokens : T;
+  decode_tables dt;
+  fill_decode_tables(&dt);
+  const decode_tables* d = &dt;
   set_threads(nthreads);
 #pragma omp parallel
   {
@@ -418,9 +457,7 @@ static void fused_moe_mx(const uint8_t* x, const uint8_t* x_scales,
 #pragma omp for schedule(dynamic, 1)
     for (int idx = 0; idx < count; ++idx) {
       const int t = tokens ? tokens[idx] : idx;
-      for (int k = 0; k < K; ++k)
-        xd[k] = orc_e4m3_to_double(x[(int64_t)t * K + k]) *
-                orc_e8m0_to_double(x_scales[(int64_t)t * KS + k / 32]);
+      dequant_x(d, x, x_scales, t, K, xd);
       for (int h = 0; h < K; ++h) acc[h] = 0.0;
       for (int j = 0; j < top_k; ++j) {
         const int e = topk_ids[(int64_t)t * top_k + j];
@@ -429,22 +466,14 @@ static void fused_moe_mx(const uint8_t* x, const uint8_t* x_scales,
         const uint8_t* S1 = w1_scales + (int64_t)e * N * KS;
         const uint8_t* W2 = w2 + (int64_t)e * K * I / (fp4 ? 2 : 1);
         const uint8_t* S2 = w2_scales + (int64_t)e * K * IS;
-        for (int n = 0; n < N; ++n) {
-          double s = 0.0;
-          for (int k = 0; k < K; ++k)
-            s += weight_code(W1, (int64_t)n * K + k, fp4) *
-                 orc_e8m0_to_double(S1[(int64_t)n * KS + k / 32]) * xd[k];
-          H[n] = s;
-        }
-        for (int i = 0; i < I; ++i) af[i] = (float)(silu(H[i]) * H[I + i]);
+        mx_route_intermediate(d, xd, W1, S1, K, N, fp4, H, af);
         orc_mx_quantize(af, I, aq, as);
-        for (int i = 0; i < I; ++i) a[i] = orc_e4m3_to_double(aq[i]) * orc_e8m0_to_double(as[i / 32]);
+        for (int i = 0; i < I; ++i) a[i] = d->e4m3[aq[i]] * d->e8m0[as[i / 32]];
         const double wgt = (double)topk_weights[(int64_t)t * top_k + j];
         for (int h = 0; h < K; ++h) {
           double s = 0.0;
           for (int i = 0; i < I; ++i)
-            s += weight_code(W2, (int64_t)h * I + i, fp4) *
-                 orc_e8m0_to_double(S2[(int64_t)h * IS + i / 32]) * a[i];
+            s += weight_code(d, W2, (int64_t)h * I + i, fp4) * d->e8m0[S2[(int64_t)h * IS + i / 32]] * a[i];
           acc[h] += wgt * s;
         }
       }
@@ -453,6 +482,44 @@ static void fused_moe_mx(const uint8_t* x, const uint8_t* x_scales,
         for (int h = 0; h < K; ++h) out_f64[(int64_t)t * K + h] = acc[h];
     }
     free(xd); free(H); free(af); free(aq); free(as); free(a); free(acc);
+  }
+}
+
+/* The fp32 SwiGLU intermediate of the mxfp8 / MXFP4 forward, per routed row,
+ * before its requant ([PFM] intro: the intermediate is requantised to mxfp8
+ * on chip; the requant itself is orc_mx_quantize).  act receives n_tokens x
+ * top_k rows of N/2 floats (token order of `tokens`, or all T tokens when it
+ * is NULL; routes in top-k order); the row of a route to an expert outside
+ * [0, E) is zero.  The same routine the forward above runs. */
+void orc_mx_intermediate(const uint8_t* x, const uint8_t* x_scales, const uint8_t* w1, const uint8_t* w1_scales,
+                         const int32_t* topk_ids, int T, int K, int N, int E, int top_k,
+                         const int32_t* tokens, int n_tokens, float* act, int nthreads, int fp4) {
+  const int I = N / 2, KS = K / 32;
+  const int count = tokens ? n_tokens : T;
+  decode_tables dt;
+  fill_decode_tables(&dt);
+  const decode_tables* d = &dt;
+  set_threads(nthreads);
+#pragma omp parallel
+  {
+    double* xd = (double*)malloc(sizeof(double) * (size_t)K);
+    double* H = (double*)malloc(sizeof(double) * (size_t)N);
+#pragma omp for schedule(dynamic, 1)
+    for (int idx = 0; idx < count; ++idx) {
+      const int t = tokens ? tokens[idx] : idx;
+      dequant_x(d, x, x_scales, t, K, xd);
+      for (int j = 0; j < top_k; ++j) {
+        float* row = act + ((int64_t)idx * top_k + j) * I;
+        const int e = topk_ids[(int64_t)t * top_k + j];
+        if (e < 0 || e >= E) {
+          for (int i = 0; i < I; ++i) row[i] = 0.0f;
+          continue;
+        }
+        mx_route_intermediate(d, xd, w1 + (int64_t)e * N * K / (fp4 ? 2 : 1), w1_scales + (int64_t)e * N * KS, K,
+                              N, fp4, H, row);
+      }
+    }
+    free(xd); free(H);
   }
 }
 

@@ -84,6 +84,13 @@ void orc_fused_moe_mxfp4(const uint8_t* x, const uint8_t* x_scales,
                          const int32_t* tokens, int n_tokens, uint16_t* out, double* out_f64,
                          int nthreads);
 
+/* The fp32 SwiGLU intermediate of the mxfp8 (fp4 = 0) or MXFP4 (fp4 = 1)
+ * forward before its requant, one row of N/2 floats per (listed token, route):
+ * act is (n_tokens or T) x top_k x N/2; rows of routes outside [0, E) are 0. */
+void orc_mx_intermediate(const uint8_t* x, const uint8_t* x_scales, const uint8_t* w1, const uint8_t* w1_scales,
+                         const int32_t* topk_ids, int T, int K, int N, int E, int top_k,
+                         const int32_t* tokens, int n_tokens, float* act, int nthreads, int fp4);
+
 /* Number of OpenMP threads a parallel region gets (for reporting). */
 int orc_max_threads(void);
 

@@ -27,6 +27,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SCRATCH = os.path.join(ROOT, "_build", "oracle_mutants")
 
+IM = "test_oracle_intermediate.py"
 F, P, R, K, Q, X = ("test_oracle_formats.py", "test_oracle_planner.py", "test_oracle_router.py",
                     "test_oracle_pack.py", "test_oracle_fp4.py", "test_oracle_ffn.py")
 
@@ -119,9 +120,9 @@ MUTANTS = [
     ("mx gate and up swapped", X, "af[i] = (float)(silu(H[i]) * H[I + i]);", "af[i] = (float)(silu(H[I + i]) * H[i]);"),
     ("mx requant from a bf16 value", X, "af[i] = (float)(silu(H[i]) * H[I + i]);",
      "af[i] = (float)orc_bf16_to_double(orc_double_to_bf16(silu(H[i]) * H[I + i]));"),
-    ("mx no requant", X, "a[i] = orc_e4m3_to_double(aq[i]) * orc_e8m0_to_double(as[i / 32]);", "a[i] = af[i];"),
-    ("mx requant scale block", X, "a[i] = orc_e4m3_to_double(aq[i]) * orc_e8m0_to_double(as[i / 32]);",
-     "a[i] = orc_e4m3_to_double(aq[i]) * orc_e8m0_to_double(as[(i / 32) ^ (IS > 1)]);"),
+    ("mx no requant", X, "a[i] = d->e4m3[aq[i]] * d->e8m0[as[i / 32]];", "a[i] = af[i];"),
+    ("mx requant scale block", X, "a[i] = d->e4m3[aq[i]] * d->e8m0[as[i / 32]];",
+     "a[i] = d->e4m3[aq[i]] * d->e8m0[as[(i / 32) ^ (IS > 1)]];"),
     ("mx x scale block", X, "x_scales[(int64_t)t * KS + k / 32]", "x_scales[(int64_t)t * KS + (k / 32 + 1) % KS]"),
     ("mx w1 scales transposed", X, "S1[(int64_t)n * KS + k / 32]", "S1[(int64_t)(k / 32) * N + n]"),
     ("mx w2 scale block", X, "S2[(int64_t)h * IS + i / 32]", "S2[(int64_t)h * IS + (i / 32 + 1) % IS]"),
@@ -135,19 +136,27 @@ MUTANTS = [
      "        if (e < 0 || e >= E) continue;\n        const uint8_t*",
      "for (int j = 0; j < top_k - (top_k > 1); ++j) {\n        const int e = topk_ids[(int64_t)t * top_k + j];\n"
      "        if (e < 0 || e >= E) continue;\n        const uint8_t*"),
-    ("mx token list ignored", X, "const int t = tokens ? tokens[idx] : idx;\n      for (int k = 0; k < K; ++k)",
-     "const int t = idx;\n      for (int k = 0; k < K; ++k)"),
+    ("mx token list ignored", X,
+     "const int t = tokens ? tokens[idx] : idx;\n      dequant_x(d, x, x_scales, t, K, xd);\n"
+     "      for (int h = 0; h < K; ++h) acc[h] = 0.0;",
+     "const int t = idx;\n      dequant_x(d, x, x_scales, t, K, xd);\n"
+     "      for (int h = 0; h < K; ++h) acc[h] = 0.0;"),
     ("mx out rounded via fp32", X, _BF16_TAIL + "xd);",
      _BF16_TAIL.replace("orc_double_to_bf16(acc[h])", "orc_double_to_bf16((float)acc[h])") + "xd);"),
-    ("fp4 nibble order", Q, "(idx & 1) ? (uint8_t)(b >> 4) : (uint8_t)(b & 0xF)",
-     "(idx & 1) ? (uint8_t)(b & 0xF) : (uint8_t)(b >> 4)"),
+    ("fp4 nibble order", Q, "(idx & 1) ? (b >> 4) : (b & 0xF)", "(idx & 1) ? (b & 0xF) : (b >> 4)"),
+    ("mx decode table off by one", X, "d->e4m3[c] = orc_e4m3_to_double((uint8_t)c);",
+     "d->e4m3[c] = orc_e4m3_to_double((uint8_t)(c ^ (c == 0x38)));"),
+    ("mx intermediate rows of the wrong route", IM, "float* row = act + ((int64_t)idx * top_k + j) * I;",
+     "float* row = act + ((int64_t)idx * top_k + (top_k - 1 - j)) * I;"),
+    ("mx intermediate of an invalid route left unwritten", IM,
+     "for (int i = 0; i < I; ++i) row[i] = 0.0f;\n          continue;", "continue;"),
 ]
 
 
 DEFAULT = ["bf16 ties away from zero", "e4m3 saturation value", "mx scale emax 7", "planner segment descending",
            "planner pads full segments", "router ties to the higher index", "shared expert weight",
            "blocked tile inner transpose", "bf16 gate and up swapped", "bf16 out rounded via fp32",
-           "mx requant scale block", "fp4 nibble order"]
+           "mx requant scale block", "fp4 nibble order", "mx intermediate rows of the wrong route"]
 
 
 def _tree(name: str) -> str:
