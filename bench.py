@@ -2,12 +2,13 @@
 """Benchmark of the fused MoE expert-FFN forward on B200.
 
 One step = the whole hot path on one batch: the routing planner (moe_align)
-followed by the fused forward (gate/up GEMM + SwiGLU, down GEMM, top-k
-weighted reduction) through the C ABI.  Default workload: the bf16 decode
-regime K=4096, N=4096 (intermediate 2048), E=256, top-6, T=256 tokens
-(block_m 128).  Inputs are synthetic and seeded (``workloads``); they are
-uploaded before the timed region.  The expert weights (12.9 GB) are larger
-than L2, so every step streams them from HBM.
+followed by the fused forward (gate/up GEMM + SwiGLU, mxfp8 requant, down
+GEMM, top-k weighted reduction) through the C ABI.  Default workload: the
+largest configuration, C4 -- mxfp8, K=7168, N=6144 (intermediate 3072),
+E=384, top-6, T=8192 tokens (block_m 128).  Inputs are synthetic and seeded
+(``workloads``); they are on the device before the timed region.  The
+expert weights (26 GB) are far larger than L2, so every step streams them
+from HBM.
 
 Printed (rank 0, one JSON line): the metric's value in TFLOP/s of routed
 FLOPs (3*T*top_k*K*N per call) for the whole job, microseconds per call,
@@ -18,10 +19,15 @@ the timed region, and the CPU oracle timed on a bounded token sample.
 
 Other rows: ``--workload C3F4`` / ``C4F4`` run the MXFP4-weight path; ``--router`` starts each step
 from router logits (``moe_route_align``); ``--router --shared S`` adds S shared experts.
+``--sweep`` prints one such line per (configuration, token count) over every workload (one GPU).
+``--peak`` measures the dense tensor-core peaks the roofline divides by (bf16 and mxfp8 GEMMs
+through torch at 8192^3) and prints them as one JSON line.
 
 Multi-GPU: ``torchrun --nproc-per-node N bench.py --gpus N``; every rank is an
-independent replica with all experts resident (no collective on the data
-path); time is the max over ranks, ``value`` the sum of all ranks' work.
+independent replica with all experts resident and its own token batch (no
+collective on the data path); time is the max over ranks, ``value`` the sum
+of all ranks' work.  The replicas hold the same expert weights: each rank
+draws E/N of the experts and the ranks all-gather them before timing.
 """
 from __future__ import annotations
 
@@ -57,8 +63,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--workload", default="C2", choices=W.workload_names())
-    ap.add_argument("--tokens", type=int, default=256)
+    ap.add_argument("--workload", default="C4", choices=W.workload_names())
+    ap.add_argument("--tokens", type=int, default=8192)
     ap.add_argument("--experts", type=int, default=0, help="override the workload's expert count (profiling)")
     ap.add_argument("--seed", type=int, default=W.DEFAULT_SEED)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU oracle baseline")
@@ -74,7 +80,17 @@ def parse_args(argv=None):
     ap.add_argument("--ctas", type=int, default=0)
     ap.add_argument("--flush-l2", action="store_true",
                     help="flush L2 between steps (automatic when the touched weights are < 4x L2)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="one line per (workload, token count) of every configuration (one GPU)")
+    ap.add_argument("--sweep-workloads", default="C1,C2,C3,C4,C5,C3F4,C4F4",
+                    help="comma-separated workloads of --sweep")
+    ap.add_argument("--peak", action="store_true", help="measure the dense bf16 and mxfp8 tensor peaks")
     args = ap.parse_args(argv)
+    if args.sweep and args.gpus != 1:
+        ap.error("--sweep runs on one GPU")
+    for w in args.sweep_workloads.split(","):
+        if w not in W.workload_names():
+            ap.error(f"--sweep-workloads: unknown workload {w}")
     if args.shared and not args.router:
         ap.error("--shared needs --router (the router appends the shared experts' routes)")
     if args.shared < 0:
@@ -85,32 +101,69 @@ def parse_args(argv=None):
 
 
 def load_peaks():
+    """The roofline's denominators: HBM copy bandwidth and the dense bf16 GEMM rate from the
+    measured MEASURED_PEAKS.json, and the dense mxfp8 GEMM rate from the committed
+    measurement in profiles/tensor_peak_mxfp8.md (``bench.py --peak`` on a B200), else 2x the bf16
+    figure (the nominal dense fp8:bf16 ratio)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+        peaks, src = {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
     except Exception:
-        return dict(FALLBACK_PEAKS), "fallback"
+        peaks, src = dict(FALLBACK_PEAKS), "fallback"
+    mx = None
+    try:
+        txt = open(os.path.join(ROOT, "profiles", "tensor_peak_mxfp8.md")).read()
+        m = re.search(r"mxfp8_tflops_burst:\s*([0-9.]+)", txt)
+        mx = float(m.group(1)) if m else None
+    except OSError:
+        pass
+    if mx:
+        peaks["mxfp8_tflops"], peaks["mxfp8_source"] = mx, "measured (profiles/tensor_peak_mxfp8.md)"
+    else:
+        peaks["mxfp8_tflops"], peaks["mxfp8_source"] = 2.0 * peaks["bf16_tflops"], "2 x bf16 (nominal ratio)"
+    return peaks, src
+
+
+def tensor_peak(sh: W.Shape, peaks: dict) -> float:
+    """Dense tensor peak (TFLOP/s) of the workload's MMA kind: bf16, or mxfp8 (also for MXFP4 weights,
+    which run on the same block-scaled f8f6f4 MMA)."""
+    return peaks["bf16_tflops"] if sh.dtype == "bf16" else peaks.get("mxfp8_tflops", 2.0 * peaks["bf16_tflops"])
 
 
 def cost_model(sh: W.Shape, topk_ids: np.ndarray, peaks: dict):
-    """Routed FLOPs, touched weight bytes and the path roofline time (s)."""
+    """Routed FLOPs, touched weight bytes, the path roofline time (s) and each kernel's
+    algorithmic bytes and FLOPs."""
     R = sh.T * sh.top_k
     flops = 3.0 * R * sh.K * sh.N
-    counts = np.bincount(topk_ids.reshape(-1)[(topk_ids.reshape(-1) >= 0) & (topk_ids.reshape(-1) < sh.E)],
-                         minlength=sh.E)
+    flat = topk_ids.reshape(-1)
+    valid = flat[(flat >= 0) & (flat < sh.E)]
+    counts = np.bincount(valid, minlength=sh.E)
     touched = int((counts > 0).sum())
+    Rv = int(valid.size)  # routes that reach an expert
     # weight bytes per value: bf16 2; mxfp8 1 + 1/32 (e8m0 per 32); MXFP4 1/2 + 1/32
     b = {"bf16": 2.0, "mxfp8": 1.0 + 1.0 / 32.0, "mxfp4": 0.5 + 1.0 / 32.0}[sh.dtype]
     bytes_w = touched * 1.5 * sh.N * sh.K * b
-    p_tc = peaks["bf16_tflops"] * (1.0 if sh.dtype == "bf16" else 2.0) * 1e12
+    p_tc = tensor_peak(sh, peaks) * 1e12
     bw = peaks["hbm_gbs"] * 1e9
     t_flop, t_hbm = flops / p_tc, bytes_w / bw
-    # gate/up phase: w1 of the touched experts, the routed rows of x, the intermediate written once
+    # bytes per activation value: bf16 2, mxfp8 1 + 1/32
     bx = 2.0 if sh.dtype == "bf16" else 1.0 + 1.0 / 32.0
-    p1_bytes = touched * sh.N * sh.K * b + R * sh.K * bx + R * sh.I * bx
-    p1_flops = 2.0 * R * sh.K * sh.N
+    kern = {
+        # gate/up: w1 of the touched experts, the routed rows of x, the intermediate written once
+        "gate_up": dict(bytes=touched * sh.N * sh.K * b + Rv * sh.K * bx + Rv * sh.I * bx,
+                        flops=2.0 * Rv * sh.K * sh.N, name="moe_p1_kernel (gather + gate/up GEMM + SwiGLU)",
+                        ncu="moe_p1_kernel"),
+        # down (+ the split-K reduction when it runs): w2, the intermediate read once, the weighted
+        # partial row of every route written once (fp32)
+        "down": dict(bytes=touched * sh.K * sh.I * b + Rv * sh.I * bx + Rv * sh.K * 4.0,
+                     flops=1.0 * Rv * sh.K * sh.N, name="moe_p2_kernel (down GEMM + routing weight)",
+                     ncu="moe_p2_kernel"),
+        # top-k reduction: every partial row read, out written, one flag per route
+        "reduce": dict(bytes=R * sh.K * 4.0 + 2.0 * sh.T * sh.K + 4.0 * R, flops=0.0,
+                       name="moe_combine_kernel (top-k weighted reduction)", ncu="moe_combine_kernel"),
+    }
     # the whole path's algorithmic HBM bytes: touched weights, x (+ its scales) read once, out written
     # once, the routing read, the planner's arrays written (sorted ids, expert ids, the padded total)
     cap = R + sh.E * (sh.block_m - 1)
@@ -118,7 +171,8 @@ def cost_model(sh: W.Shape, topk_ids: np.ndarray, peaks: dict):
             "plan": 4.0 * cap + 4.0 * ((cap + sh.block_m - 1) // sh.block_m) + 4.0}
     return dict(R=R, flops=flops, touched=touched, bytes_w=bytes_w, t_flop=t_flop, t_hbm=t_hbm,
                 t_roof=max(t_flop, t_hbm), bound="tensor" if t_flop > t_hbm else "hbm", p_tc=p_tc, bw=bw,
-                p1_bytes=p1_bytes, p1_flops=p1_flops, bytes_full=sum(full.values()), bytes_parts=full)
+                p1_bytes=kern["gate_up"]["bytes"], p1_flops=kern["gate_up"]["flops"], kernels=kern,
+                bytes_full=sum(full.values()), bytes_parts=full)
 
 
 class ClockSampler:
@@ -271,11 +325,97 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+def upload_weights(sh: W.Shape, inp: dict, dev) -> dict:
+    """Host expert weights (the generator's arrays) to the device; e8m0 scales packed blocked."""
+    import torch
+
+    import mixture_experts_ffn_planner_b200 as moe
+
+    def up(a, dtype=None):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        return (t.view(dtype) if dtype is not None else t).to(dev)
+
+    if sh.dtype == "bf16":
+        return dict(w1=up(inp["w1"], torch.bfloat16), w2=up(inp["w2"], torch.bfloat16), s1=None, s2=None)
+    return dict(w1=up(inp["w1"]), w2=up(inp["w2"]), s1=moe.pack_scales_blocked(up(inp["w1_scales"])),
+                s2=moe.pack_scales_blocked(up(inp["w2_scales"])))
+
+
+def _expert_arrays(sh: W.Shape, which: str, e: int, seed: int):
+    """One expert's weights as the caller hands them over: bf16 bits, or (codes, row-major scales)."""
+    v = W.expert_f32(sh, which, e, seed)
+    if sh.dtype == "bf16":
+        return W.f32_to_bf16_bits(v), None
+    return W.mx_quantize_fp4(v) if sh.dtype == "mxfp4" else W.mx_quantize_inputs(v)
+
+
+def device_weights(sh: W.Shape, seed: int, dev, world: int = 1, rank: int = 0, dist=None, threads: int = 0) -> dict:
+    """The workload's expert weights drawn expert by expert straight into device memory (no host copy
+    of the whole set).  With several ranks each draws E/world of the experts and the ranks all-gather
+    them, so every replica holds the same weights and the draws are split between the ranks."""
+    import concurrent.futures as cf
+
+    import torch
+
+    import mixture_experts_ffn_planner_b200 as moe
+
+    pack = 2 if sh.dtype == "mxfp4" else 1
+    split = world > 1 and sh.E % world == 0
+    lo, hi = (rank * sh.E // world, (rank + 1) * sh.E // world) if split else (0, sh.E)
+    wdt = torch.uint16 if sh.dtype == "bf16" else torch.uint8
+    dims = {"w1": (sh.N, sh.K), "w2": (sh.K, sh.I)}
+    out = {}
+    for which, (rows, cols) in dims.items():
+        loc = torch.empty((hi - lo, rows, cols // pack), dtype=wdt, device=dev)
+        sc = None if sh.dtype == "bf16" else torch.empty((hi - lo, rows, cols // 32), dtype=torch.uint8, device=dev)
+
+        def job(e):
+            v, s_ = _expert_arrays(sh, which, e, seed)
+            loc[e - lo].copy_(torch.from_numpy(v))
+            if sc is not None:
+                sc[e - lo].copy_(torch.from_numpy(s_))
+        n = threads if threads > 0 else max(1, min(32, (os.cpu_count() or 1) // max(1, world)))
+        with cf.ThreadPoolExecutor(n) as ex:
+            list(ex.map(job, range(lo, hi)))
+        if split:
+            full = torch.empty((sh.E,) + tuple(loc.shape[1:]), dtype=wdt, device=dev)
+            dist.all_gather_into_tensor(full, loc)
+            loc = full
+            if sc is not None:
+                fs = torch.empty((sh.E,) + tuple(sc.shape[1:]), dtype=torch.uint8, device=dev)
+                dist.all_gather_into_tensor(fs, sc)
+                sc = fs
+        out[which] = loc.view(torch.bfloat16) if sh.dtype == "bf16" else loc
+        out["s1" if which == "w1" else "s2"] = None if sc is None else moe.pack_scales_blocked(sc)
+    return out
+
+
+def step_inputs(sh: W.Shape, seed: int) -> dict:
+    """A step's token batch: x (bf16 bits, or e4m3 codes + e8m0 scales) and the routing."""
+    ids, tw = W.routing(sh, seed)
+    d = dict(topk_ids=ids, topk_weights=tw)
+    if sh.dtype == "bf16":
+        d["x"] = W.f32_to_bf16_bits(W.x_f32(sh, seed))
+    else:
+        d["x"], d["x_scales"] = W.mx_quantize_inputs(W.x_f32(sh, seed))
+    return d
+
+
+def host_weights(sh: W.Shape, seed: int) -> dict:
+    """The expert weights as host arrays (kept for the CPU oracle legs)."""
+    if sh.dtype == "bf16":
+        return dict(w1=W.bf16_weights(sh, "w1", seed), w2=W.bf16_weights(sh, "w2", seed))
+    wq = W.mxfp4_weights if sh.dtype == "mxfp4" else W.mxfp8_weights
+    w1, s1 = wq(sh, "w1", seed)
+    w2, s2 = wq(sh, "w2", seed)
+    return dict(w1=w1, w1_scales=s1, w2=w2, w2_scales=s2)
+
+
 class Problem:
     """Device-resident inputs of one workload and one step of the hot path."""
 
     def __init__(self, sh: W.Shape, inp: dict, dev, stages: int = 0, ctas: int = 0, router: bool = False,
-                 n_shared: int = 0):
+                 n_shared: int = 0, weights: dict | None = None):
         import torch
 
         import mixture_experts_ffn_planner_b200 as moe
@@ -302,23 +442,23 @@ class Problem:
         self.e_ids = torch.empty((cap + bm - 1) // bm, dtype=torch.int32, device=dev)
         self.ntpp = torch.empty(1, dtype=torch.int32, device=dev)
         self.out = torch.empty((sh.T, sh.K), dtype=torch.bfloat16, device=dev)
+        if weights is None:
+            weights = upload_weights(sh, inp, dev)
+        self.w1, self.w2, self.s1, self.s2 = weights["w1"], weights["w2"], weights["s1"], weights["s2"]
         if sh.dtype == "bf16":
             self.x = up(inp["x"], torch.bfloat16)
-            self.w1, self.w2 = up(inp["w1"], torch.bfloat16), up(inp["w2"], torch.bfloat16)
-            self.xs = self.s1 = self.s2 = None
+            self.xs = None
             dt = moe.DTYPE_BF16
         else:
-            self.x, self.xs, self.w1, self.w2 = up(inp["x"]), up(inp["x_scales"]), up(inp["w1"]), up(inp["w2"])
-            self.s1 = moe.pack_scales_blocked(up(inp["w1_scales"]))
-            self.s2 = moe.pack_scales_blocked(up(inp["w2_scales"]))
+            self.x, self.xs = up(inp["x"]), up(inp["x_scales"])
             dt = moe.DTYPE_MXFP4 if sh.dtype == "mxfp4" else moe.DTYPE_MXFP8
         self.ws = torch.empty(moe.moe_workspace_bytes(dt, sh.T, sh.K, sh.N, sh.E + n_shared, sh.top_k + n_shared, bm),
                               dtype=torch.uint8, device=dev)
         self.plain = moe.Tuning(stages, ctas, None)
         self.stages, self.ctas = stages, ctas
         # planner, gate/up phase, split-K reduction, down phase, combine (+ the router kernel for
-        # batches of more than 128 tokens on the router path)
-        self.launches_per_step = 5 + (1 if router and sh.T > 128 else 0)
+        # batches of more than 32 tokens on the router path)
+        self.launches_per_step = 5 + (1 if router and sh.T > 32 else 0)
 
     def fused(self, tune):
         m = self.moe
@@ -475,22 +615,29 @@ def measure_e2e(prob: Problem, steps: int, barrier=None):
     return e0.elapsed_time(e1), h2d, d2h
 
 
-def roofline_of_p1(sh: W.Shape, cm: dict, p1_ms: float, peaks: dict, peak_src: str):
-    p1_s = p1_ms * 1e-3
+def roofline_of(sh: W.Shape, cm: dict, m: dict, peaks: dict, peak_src: str):
+    """Roofline of the kernel with the longest device time in the step (pass 2 phase events):
+    its algorithmic bytes (or FLOPs) per launch over its measured duration, against the measured
+    HBM copy bandwidth (or the tensor peak of its MMA kind), whichever bound is slower."""
+    phase_ms = {"gate_up": m["p1_ms"], "down": m["p2_ms"], "reduce": m["cb_ms"]}
+    which = max(phase_ms, key=phase_ms.get)
+    k = cm["kernels"][which]
+    sec = phase_ms[which] * 1e-3
     tag = f"{sh.name}_T{sh.T}"
-    name = "moe_p1_kernel (gather + gate/up GEMM + SwiGLU)"
-    if cm["p1_flops"] / cm["p_tc"] <= cm["p1_bytes"] / cm["bw"]:
-        gbs = cm["p1_bytes"] / p1_s / 1e9
-        return {"kernel": name, "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": gbs / peaks["hbm_gbs"], "traffic": kernel_traffic("moe_p1_kernel", tag),
-                "peak_source": f"{peak_src} hbm_gbs", "algorithmic_bytes_per_launch": cm["p1_bytes"],
-                "us_per_launch": p1_ms * 1e3}
-    pk = peaks["bf16_tflops"] * (1.0 if sh.dtype == "bf16" else 2.0)
-    tf = cm["p1_flops"] / p1_s / 1e12
-    return {"kernel": name, "bound": "tensor", "achieved": tf, "peak": pk, "unit": "TFLOP/s", "frac": tf / pk,
-            "traffic": kernel_traffic("moe_p1_kernel", tag),
-            "peak_source": f"{peak_src} bf16_tflops" + ("" if sh.dtype == "bf16" else " x 2 (fp8:bf16 nominal)"),
-            "algorithmic_flops_per_launch": cm["p1_flops"], "us_per_launch": p1_ms * 1e3}
+    pk_tc = tensor_peak(sh, peaks)
+    base = {"kernel": k["name"], "phase": which, "us_per_launch": phase_ms[which] * 1e3,
+            "share_of_step": phase_ms[which] / max(sum(phase_ms.values()) + m["plan_ms"], 1e-12),
+            "traffic": kernel_traffic(k["ncu"], tag)}
+    if k["flops"] / (pk_tc * 1e12) <= k["bytes"] / cm["bw"]:
+        gbs = k["bytes"] / sec / 1e9
+        return {**base, "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
+                "algorithmic_bytes_per_launch": k["bytes"]}
+    tf = k["flops"] / sec / 1e12
+    src = f"{peak_src} bf16_tflops" if sh.dtype == "bf16" else \
+        f"mxfp8 dense: {peaks.get('mxfp8_source', '2 x bf16 (nominal ratio)')}"
+    return {**base, "bound": "tensor", "achieved": tf, "peak": pk_tc, "unit": "TFLOP/s", "frac": tf / pk_tc,
+            "peak_source": src, "algorithmic_flops_per_launch": k["flops"]}
 
 
 def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
@@ -513,10 +660,12 @@ def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
                           "routed_gflop": cm["flops"] / 1e9, "touched_weight_gb": cm["bytes_w"] / 1e9,
                           "algorithmic_hbm_gb": cm["bytes_full"] / 1e9,
                           "algorithmic_hbm_parts_gb": {k: v / 1e9 for k, v in cm["bytes_parts"].items()},
-                          "peaks": peak_src},
+                          "peaks": peak_src, "tensor_peak_tflops": tensor_peak(sh, peaks),
+                          **({} if sh.dtype == "bf16" else
+                             {"mxfp8_peak_source": peaks.get("mxfp8_source", "2 x bf16 (nominal ratio)")})},
         "phase_us": {"planner": m["plan_ms"] * 1e3, "gate_up": m["p1_ms"] * 1e3, "down": m["p2_ms"] * 1e3,
                      "reduce": m["cb_ms"] * 1e3},
-        "roofline": roofline_of_p1(sh, cm, m["p1_ms"], peaks, peak_src),
+        "roofline": roofline_of(sh, cm, m, peaks, peak_src),
         "gpu_launches": m["launches"],
         "clocks": m["clocks"],
         **({"warm": {"us_per_call": m["warm_ms_step"] * 1e3,
@@ -542,44 +691,36 @@ def whole_job_tflops(flops_per_rank: float, world: int, ms_per_step: float) -> f
     return world * flops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
-def run_b200(args):
-    import torch
-    import torch.distributed as dist
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    if world > 1:
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    barrier = dist.barrier if world > 1 else None
-    dev = torch.device("cuda", local)
-    peaks, peak_src = load_peaks()
-
-    sh = W.shape(args.workload, args.tokens, **({"E": args.experts} if args.experts else {}))
+def _setup_inputs(sh: W.Shape, args, rank: int, world: int, dist, dev, need_host: bool):
+    """(shape with the shared experts, host inputs, device weights) of one workload.  Replicas share
+    the expert weights (seed) and draw their own token batch (seed + rank)."""
+    seed_w, seed_x = args.seed, args.seed + rank
+    sh_w = dataclasses.replace(sh, E=sh.E + args.shared, top_k=sh.top_k + args.shared) if args.shared else sh
+    inp = step_inputs(sh, seed_x)
     if args.shared:
-        # weights of the routed experts followed by the shared ones
-        sh_w = dataclasses.replace(sh, E=sh.E + args.shared, top_k=sh.top_k + args.shared)
-        inp = W.inputs(sh_w, seed=args.seed + rank)
         # the generator's routing over the routed experts, then the shared routes (cost model and
         # CPU baseline; the timed step routes from logits on the GPU)
-        ids, tw = W.routing(sh, seed=args.seed + rank)
         shared_ids = np.broadcast_to(np.arange(sh.E, sh.E + args.shared, dtype=np.int32), (sh.T, args.shared))
-        inp["topk_ids"] = np.ascontiguousarray(np.concatenate([ids, shared_ids], axis=1))
+        inp["topk_ids"] = np.ascontiguousarray(np.concatenate([inp["topk_ids"], shared_ids], axis=1))
         inp["topk_weights"] = np.ascontiguousarray(
-            np.concatenate([tw, np.ones((sh.T, args.shared), np.float32)], axis=1))
-    else:
-        inp = W.inputs(sh, seed=args.seed + rank)  # every replica gets its own batch
+            np.concatenate([inp["topk_weights"], np.ones((sh.T, args.shared), np.float32)], axis=1))
     if args.router:
-        inp["router_logits"], inp["router_bias"] = W.router_logits(sh, seed=args.seed + rank)
-    cm = cost_model(sh_w if args.shared else sh, inp["topk_ids"], peaks)
-    prob = Problem(sh, inp, dev, args.stages, args.ctas, router=args.router, n_shared=args.shared)
+        inp["router_logits"], inp["router_bias"] = W.router_logits(sh, seed=seed_x)
+    if need_host:
+        inp.update(host_weights(sh_w, seed_w))
+        weights = upload_weights(sh_w, inp, dev)
+    else:
+        weights = device_weights(sh_w, seed_w, dev, world, rank, dist)
+    return sh_w, inp, weights
+
+
+def bench_point(sh: W.Shape, sh_w: W.Shape, inp: dict, weights: dict, args, world: int, rank: int, local: int,
+                dist, dev, peaks, peak_src, barrier, cpu_seconds: float):
+    """Measures one workload and returns its JSON line (rank 0 prints it)."""
+    cm = cost_model(sh_w, inp["topk_ids"], peaks)
+    prob = Problem(sh, inp, dev, args.stages, args.ctas, router=args.router, n_shared=args.shared, weights=weights)
     flush = args.flush_l2 or cm["bytes_w"] < 4 * 126e6
     m = measure(prob, args.steps, args.warmup, flush_l2=flush, barrier=barrier, local=local)
-
     m["ms_step"] = max_over_ranks(m["ms_step"], world, dist, dev)
     line = result_line(sh, cm, m, world, args.steps, args.warmup, peaks, peak_src, flush)
     if args.router:
@@ -593,9 +734,38 @@ def run_b200(args):
                        "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                        "us_per_call": 1e3 * ems / args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, thr, desc, spent = oracle_sample_rate(sh, inp, args.cpu_seconds, args.seed, args.cpu_threads)
+        rate, thr, desc, spent = oracle_sample_rate(sh_w, inp, cpu_seconds, args.seed, args.cpu_threads)
         line["cpu_baseline"] = {"value": rate, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                                 "sample": desc, "seconds": spent}
+    del prob
+    return line
+
+
+def _init(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local, dist, torch.device("cuda", local)
+
+
+def run_b200(args):
+    world, rank, local, dist, dev = _init(args)
+    barrier = dist.barrier if world > 1 else None
+    peaks, peak_src = load_peaks()
+    sh = W.shape(args.workload, args.tokens, **({"E": args.experts} if args.experts else {}))
+    need_host = rank == 0 and world == 1 and not args.no_cpu_baseline
+    sh_w, inp, weights = _setup_inputs(sh, args, rank, world, dist, dev, need_host)
+    line = bench_point(sh, sh_w, inp, weights, args, world, rank, local, dist, dev, peaks, peak_src, barrier,
+                       args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -604,10 +774,106 @@ def run_b200(args):
     return 0
 
 
+def run_sweep(args):
+    """One line per (workload, token count) of the chosen configurations, on one GPU; every line
+    carries its own clock record, path roofline, dominant-kernel roofline and CPU oracle sample
+    (a shorter budget per line: --cpu-seconds / 5)."""
+    import torch
+
+    world, rank, local, dist, dev = _init(args)
+    peaks, peak_src = load_peaks()
+    for name in args.sweep_workloads.split(","):
+        base = W.shape(name)
+        weights = inp_w = None
+        for T in W.token_counts(name):
+            sh = W.shape(name, T)
+            if weights is None:
+                need_host = not args.no_cpu_baseline
+                sh_w, inp, weights = _setup_inputs(sh, args, rank, world, dist, dev, need_host)
+                inp_w = {k: v for k, v in inp.items() if k.startswith("w")}
+            else:
+                sh_w = sh
+                inp = dict(step_inputs(sh, args.seed + rank), **inp_w)
+                if args.router:
+                    inp["router_logits"], inp["router_bias"] = W.router_logits(sh, seed=args.seed + rank)
+            line = bench_point(sh, sh_w, inp, weights, args, world, rank, local, dist, dev, peaks, peak_src, None,
+                               max(1.0, args.cpu_seconds / 5))
+            line["sweep"] = f"{name} T={T}"
+            print(json.dumps(line), flush=True)
+        del weights, inp_w, base
+        torch.cuda.empty_cache()
+    return 0
+
+
+def run_peak(args):
+    """Dense tensor-core peaks on this GPU: a bf16 GEMM (torch.matmul) and an mxfp8 GEMM
+    (torch.nn.functional.scaled_mm, e4m3 operands with one e8m0 scale per 32 along K), both
+    M = N = K = 8192, as a burst (best of 20 timed calls) and sustained (back to back for ~4 s)."""
+    import torch
+    import torch.nn.functional as F
+
+    _, _, local, _, dev = _init(args)
+    n = 8192
+    flop = 2.0 * n ** 3
+    a16 = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
+    b16 = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
+    a8 = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    b8 = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+    ones = torch.full((n * n // 32,), 127, dtype=torch.uint8, device=dev).view(torch.float8_e8m0fnu)
+
+    def mx():
+        return F.scaled_mm(a8, b8.t(), ones, F.ScalingType.BlockWise1x32, ones, F.ScalingType.BlockWise1x32,
+                           swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                           output_dtype=torch.bfloat16)
+
+    def bf():
+        return a16 @ b16
+
+    res = {"metric": "dense tensor-core peak", "M=N=K": n}
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    for name, fn in (("bf16", bf), ("mxfp8", mx)):
+        try:
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            best = float("inf")
+            for _ in range(20):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                best = min(best, e0.elapsed_time(e1))
+            t0 = time.perf_counter()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            calls = 0
+            while time.perf_counter() - t0 < 4.0:
+                for _ in range(20):
+                    fn()
+                calls += 20
+                torch.cuda.synchronize()
+            e1.record()
+            torch.cuda.synchronize()
+            res[f"{name}_tflops_burst"] = flop / (best * 1e-3) / 1e12
+            res[f"{name}_tflops_sustained"] = flop * calls / (e0.elapsed_time(e1) * 1e-3) / 1e12
+        except Exception as exc:  # an operand type this torch build cannot run
+            res[f"{name}_error"] = f"{type(exc).__name__}: {exc}"[:300]
+    res["clocks"] = clocks.stop()
+    print(json.dumps(res), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.peak:
+        return run_peak(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_b200(args)
 
 

@@ -168,10 +168,16 @@ typedef struct moe_tuning {
   int stages;   /* shared-memory pipeline depth of the GEMM phases        */
   int num_ctas; /* persistent CTAs per phase (default: one per SM)        */
   /* Timing hook: if non-NULL, four caller-created cudaEvent_t handles that
-   * are recorded on `stream` before the gate/up phase, between it and the
-   * down phase, between the down phase and the reduction, and after the
-   * reduction. */
+   * are recorded on `stream` before the gate/up phase, between it (with the
+   * split-K reduction after it) and the down phase, between the down phase
+   * and the top-k reduction, and after the reduction. */
   void* const* phase_events;
+  /* Limit, in ns of the GPU's global timer, of every bounded wait inside the
+   * fused kernels (0: the default of 2 s).  A wait that runs out makes its
+   * kernel stop, and moe_device_status() then reports MOE_ERR_TIMEOUT; the
+   * call's out is undefined.  A tiny limit is a way to exercise that path;
+   * it has no other use. */
+  long long wait_timeout_ns;
 } moe_tuning;
 
 /* ------------------------------------------------------------------------

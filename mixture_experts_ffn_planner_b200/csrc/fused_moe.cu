@@ -33,9 +33,7 @@
 //            the block's intermediate rows (TMA, one 128-row box for blocks of
 //            at least 64 rows), B = 256 rows of w2[e] (TMA, one box),
 //            D in TMEM; each epilogue thread scales its row by the routing
-//            weight and writes one row segment per route (fp32 on the bf16
-//            path; bf16 on the mxfp8 path, whose tolerance leaves room for
-//            the extra rounding).
+//            weight and writes one fp32 row segment per route.
 //   combine  out[t] = bf16(sum over the token's routes, in route order), a
 //            deterministic HBM-bound pass.
 // The weight tiles are streamed once per unit through a multi-stage shared
@@ -68,11 +66,23 @@ constexpr int kTH = 256;          // output features per down unit (MMA N)
 constexpr int kRowBytes = 128;    // bytes of one operand row per pipeline stage
 constexpr int kSfTileBytes = 512; // one blocked scale tile: 128 rows x 4 scales
 constexpr int kSmemLimit = 232448;  // 227 KB of dynamic shared memory per CTA
+// L2 prefetch budgets of small calls (the L2 holds 126 MB): all expert
+// weights when they fit kPrefetchAllBytes; else the down phase's w2 tiles of
+// the planner blocks when they fit kPrefetchW2Bytes.
+constexpr int64_t kPrefetchAllBytes = int64_t(40) << 20;
+constexpr int64_t kPrefetchW2Bytes = int64_t(48) << 20;
 
 // TMEM column map: accumulators first; on the mxfp8 path (one accumulator)
-// the scale factors follow it.
-constexpr uint32_t kSfaCol = 256;   // 4 columns: 128 rows of A
-constexpr uint32_t kSfbCol = 260;   // 8 columns: 256 rows of B
+// the scale factors follow it, one set of 12 columns per pipeline stage (4
+// for the 128 rows of A, 8 for the 256 rows of B).  A stage's scales are
+// copied into its own columns, so the copy never waits for the MMAs of the
+// previous stage, which still read theirs; a set is rewritten only after the
+// stage's MMAs completed (the stage was released through its empty barrier).
+constexpr uint32_t kSfCol0 = 256;
+constexpr uint32_t kSfColsPerStage = 12;
+constexpr int kMaxStages = 8;  // 256 + 8 * 12 <= 512 TMEM columns
+__device__ __forceinline__ uint32_t sfa_col(int s) { return kSfCol0 + kSfColsPerStage * static_cast<uint32_t>(s); }
+__device__ __forceinline__ uint32_t sfb_col(int s) { return sfa_col(s) + 4; }
 
 constexpr int kEpiWarps = 8;
 constexpr int kGatherWarps = 4;
@@ -114,6 +124,18 @@ struct P1Params {
   int n_jt;                 // ceil(I / 128): work units per planner block
   int stages, stage_bytes;
   int off_b, off_sf;        // stage offsets of the B tile and of the scale tiles
+  unsigned long long wait_ns;  // limit of every bounded wait
+  // L2 prefetch for small calls (0 / null: none).  pf_all: the byte ranges of
+  // all expert weights (and scales), fetched while the planner still runs;
+  // otherwise, when the blocks' down-projection tiles fit pf_w2_budget bytes,
+  // the w2 tiles the down phase will read, fetched while this phase computes.
+  const uint8_t* pf_src[4];
+  int64_t pf_bytes[4];
+  int pf_all;
+  const uint8_t* w2;        // (E, K, N/2) codes: w2_row_bytes per row
+  const uint8_t* w2_sf;     // blocked scales of w2 (mxfp8), or null
+  int64_t w2_row_bytes;
+  int64_t pf_w2_budget;
 };
 
 struct P2Params {
@@ -123,7 +145,7 @@ struct P2Params {
   const int32_t* expert_ids;
   const int32_t* ntpp;
   const float* topk_w;
-  void* yw;                 // (R, K) weighted down-projection rows: fp32 (bf16 path) or bf16 (mxfp8 path)
+  void* yw;                 // (R, K) weighted down-projection rows, fp32
   int32_t* flags;
   int* status;
   int K, I, E, top_k, bm, R;
@@ -131,10 +153,12 @@ struct P2Params {
   int w_reuse;
   int n_ht;                 // ceil(K / 256): work units per planner block
   int n_kc;                 // K-chunks of the down GEMM
+  int nsplit2;              // small calls: the down GEMM's N/2 range is split this many ways
   int a_full;               // the stage's A region holds 128 rows
   int w_fp4;                // weights are MXFP4 (as in the gate/up phase)
   int stages, stage_bytes;
   int off_b, off_sf;
+  unsigned long long wait_ns;
 };
 
 // Per-unit facts every warp role derives the same way (warp-collective).
@@ -294,6 +318,16 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     tmem_alloc(tmem_base_sm, 512);
     tmem_relinquish();
   }
+  if (warp == 2 && lane == 0 && p.pf_all) {
+    // small expert set: this CTA's share of every weight byte range goes to
+    // L2 now, while the planner runs (the touched experts are not known yet)
+    for (int a = 0; a < 4; ++a) {
+      const int64_t n16 = p.pf_bytes[a] / 16;
+      const int64_t lo = n16 * blockIdx.x / gridDim.x * 16, hi = n16 * (blockIdx.x + 1) / gridDim.x * 16;
+      for (int64_t o = lo; o < hi; o += 32768)
+        prefetch_l2(p.pf_src[a] + o, static_cast<uint32_t>(hi - o < 32768 ? hi - o : 32768));
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -358,7 +392,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       const int up_row = bi.e * p.N + p.I + j * kTI;
       for (int kc = k0; kc < k1; ++kc) {
         if (lane == 0) {
-          ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
+          ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, p.wait_ns);
           if (ok) {
             uint8_t* st = stage_ptr(s);
             mbar_arrive_expect_tx(&full[s], tx);
@@ -396,14 +430,14 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       if (k0 == k1) continue;
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
-      if (lane == 0) ok = mbar_wait(&acc_empty[buf], acc_ph ^ 1u, abort_flag, p.status);
+      if (lane == 0) ok = mbar_wait(&acc_empty[buf], acc_ph ^ 1u, abort_flag, p.status, p.wait_ns);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
       const uint32_t d = tbase + static_cast<uint32_t>(buf) * 256u;
       for (int kc = k0; kc < k1; ++kc) {
         if (lane == 0) {
-          ok = mbar_wait(&full[s], ph, abort_flag, p.status);
+          ok = mbar_wait(&full[s], ph, abort_flag, p.status, p.wait_ns);
           if (ok) {
             tc_fence_after();
             // the token rows (and scales) arrived through cp.async (generic
@@ -413,9 +447,9 @@ __global__ void __launch_bounds__(kP1Threads, 1)
             const uint64_t ad = sdesc_sw128(smem_u32(st));
             const uint64_t bd = sdesc_sw128(smem_u32(st + p.off_b));
             if (kFp8) {
-              tc_cp_32x128b_x4(tbase + kSfaCol, sdesc_sf(smem_u32(st + p.off_sf)));
-              tc_cp_32x128b_x4(tbase + kSfbCol, sdesc_sf(smem_u32(st + p.off_sf + kSfTileBytes)));
-              tc_cp_32x128b_x4(tbase + kSfbCol + 4, sdesc_sf(smem_u32(st + p.off_sf + 2 * kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + sfa_col(s), sdesc_sf(smem_u32(st + p.off_sf)));
+              tc_cp_32x128b_x4(tbase + sfb_col(s), sdesc_sf(smem_u32(st + p.off_sf + kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + sfb_col(s) + 4, sdesc_sf(smem_u32(st + p.off_sf + 2 * kSfTileBytes)));
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -424,7 +458,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
               if (kFp8) {
                 const uint32_t sfid = static_cast<uint32_t>(kk) << 30;
                 mma_mxf8(d, ad + step, bd + step, idesc_mxf8(kM, 256, kk, kk, p.w_fp4 ? kFmtE2M1 : kFmtE4M3),
-                         (tbase + kSfaCol) | sfid, (tbase + kSfbCol) | sfid, acc);
+                         (tbase + sfa_col(s)) | sfid, (tbase + sfb_col(s)) | sfid, acc);
               } else {
                 mma_f16(d, ad + step, bd + step, kIdesc, acc);
               }
@@ -486,7 +520,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
         if (r < bi.nend && row_valid(bi, r)) sf_src = p.x_sf + static_cast<int64_t>(pf_id(cur, g) / p.top_k) * KS;
       }
       for (int kc = k0; kc < k1; ++kc) {
-        if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
+        if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, p.wait_ns);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         const uint32_t abase = smem_u32(stage_ptr(s));
@@ -500,6 +534,25 @@ __global__ void __launch_bounds__(kP1Threads, 1)
     }
   } else {
     // ------------------------------------------------ epilogue (8 warps)
+    if (warp == kP1FirstEpi && lane == 0 && !p.pf_all && p.pf_w2_budget > 0) {
+      // Small calls: while this phase computes, pull into L2 the w2 tiles
+      // (256 rows each) the down phase's units will read, this CTA's share
+      // of the down phase's unit list, unless they exceed the budget.
+      const int n_ht2 = (p.K + kTH - 1) / kTH;
+      if (static_cast<int64_t>(n_blocks) * p.K * p.w2_row_bytes <= p.pf_w2_budget) {
+        const int KT2 = p.I / 128, MT2 = p.K / 128;
+        for (int u = blockIdx.x; u < n_blocks * n_ht2; u += gridDim.x) {
+          const int e = __ldg(p.expert_ids + u / n_ht2), ht = u % n_ht2;
+          if (e < 0 || e >= p.E) continue;
+          const int rows = min(kTH, p.K - ht * kTH);
+          prefetch_l2(p.w2 + (static_cast<int64_t>(e) * p.K + ht * kTH) * p.w2_row_bytes,
+                      static_cast<uint32_t>(rows * p.w2_row_bytes));
+          if (p.w2_sf)
+            prefetch_l2(p.w2_sf + ((static_cast<int64_t>(e) * MT2 + ht * (kTH / 128)) * KT2) * kSfTileBytes,
+                        static_cast<uint32_t>(rows / 128 * KT2 * kSfTileBytes));
+        }
+      }
+    }
     // Warp w reads TMEM lane quadrant w % 4 (rows 32q..32q+31, one per
     // thread) and intermediate columns [64h, 64h + 64) of the unit's tile.
     const int q = warp & 3;
@@ -520,7 +573,7 @@ __global__ void __launch_bounds__(kP1Threads, 1)
       if (k0 == k1) continue;
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
-      ok = mbar_wait(&acc_full[buf], acc_ph, abort_flag, p.status);
+      ok = mbar_wait(&acc_full[buf], acc_ph, abort_flag, p.status, p.wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -754,6 +807,9 @@ __global__ void __launch_bounds__(kP2Threads, 1)
   constexpr int TH = kTH;
   const int n_ht = p.n_ht;
   const int n_units = n_blocks * n_ht;
+  // work items: (unit, split of the N/2 contraction); without splitting an item is a unit
+  const int S2 = p.nsplit2;
+  const int n_items = n_units * S2, per_block = n_ht * S2;
   constexpr int kKC = kFp8 ? 128 : 64;
   auto stage_ptr = [&](int s) { return smem + static_cast<size_t>(s) * p.stage_bytes; };
 
@@ -765,11 +821,12 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_ht, p.bm);
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int b = u / n_ht, ht = u - (u / n_ht) * n_ht;
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_items, per_block, p.bm);
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      const int u = w / S2, b = u / n_ht, ht = u - (u / n_ht) * n_ht;
+      const int k0 = (w - u * S2) * p.n_kc / S2, k1 = (w - u * S2 + 1) * p.n_kc / S2;
       const BlockPf cur = pf;
-      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_ht, p.bm);
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, w + gridDim.x, n_items, per_block, p.bm);
       const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
       const int nb = min(TH, p.K - ht * TH) / 128;  // 128-row pieces of this feature tile
@@ -782,9 +839,9 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       const int a_rows = big_a ? 128 : bi.n16;
       const uint32_t w_row_bytes = p.w_fp4 ? kRowBytes / 2 : kRowBytes;  // packed MXFP4 rows
       const uint32_t tx = nb * 128 * w_row_bytes + a_rows * kRowBytes + (kFp8 ? (1 + nb) * kSfTileBytes : 0);
-      for (int kc = 0; kc < p.n_kc; ++kc) {
+      for (int kc = k0; kc < k1; ++kc) {
         if (lane == 0) {
-          ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status);
+          ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag, p.status, p.wait_ns);
           if (ok) {
             uint8_t* st = stage_ptr(s);
             mbar_arrive_expect_tx(&full[s], tx);
@@ -819,42 +876,43 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     uint32_t ph = 0;
     int acc_it = 0;
     bool ok = true;
-    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_ht, p.bm);
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int ht = u - (u / n_ht) * n_ht;
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_items, per_block, p.bm);
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      const int u = w / S2, ht = u - (u / n_ht) * n_ht;
+      const int k0 = (w - u * S2) * p.n_kc / S2, k1 = (w - u * S2 + 1) * p.n_kc / S2;
       const BlockPf cur = pf;
-      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_ht, p.bm);
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, w + gridDim.x, n_items, per_block, p.bm);
       const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
       const int nn = min(TH, p.K - ht * TH);
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
-      if (lane == 0) ok = mbar_wait(&acc_empty[buf], acc_ph ^ 1u, abort_flag, p.status);
+      if (lane == 0) ok = mbar_wait(&acc_empty[buf], acc_ph ^ 1u, abort_flag, p.status, p.wait_ns);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
       const uint32_t d = tbase + static_cast<uint32_t>(buf) * 256u;
-      for (int kc = 0; kc < p.n_kc; ++kc) {
+      for (int kc = k0; kc < k1; ++kc) {
         if (lane == 0) {
-          ok = mbar_wait(&full[s], ph, abort_flag, p.status);
+          ok = mbar_wait(&full[s], ph, abort_flag, p.status, p.wait_ns);
           if (ok) {
             tc_fence_after();
             uint8_t* st = stage_ptr(s);
             const uint64_t ad = sdesc_sw128(smem_u32(st));
             const uint64_t bd = sdesc_sw128(smem_u32(st + p.off_b));
             if (kFp8) {
-              tc_cp_32x128b_x4(tbase + kSfaCol, sdesc_sf(smem_u32(st + p.off_sf)));
-              tc_cp_32x128b_x4(tbase + kSfbCol, sdesc_sf(smem_u32(st + p.off_sf + kSfTileBytes)));
-              tc_cp_32x128b_x4(tbase + kSfbCol + 4, sdesc_sf(smem_u32(st + p.off_sf + 2 * kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + sfa_col(s), sdesc_sf(smem_u32(st + p.off_sf)));
+              tc_cp_32x128b_x4(tbase + sfb_col(s), sdesc_sf(smem_u32(st + p.off_sf + kSfTileBytes)));
+              tc_cp_32x128b_x4(tbase + sfb_col(s) + 4, sdesc_sf(smem_u32(st + p.off_sf + 2 * kSfTileBytes)));
             }
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t acc = (kc | kk) != 0;
+              const uint32_t acc = (kc != k0 || kk != 0) ? 1u : 0u;
               const uint64_t step = static_cast<uint64_t>(2 * kk);
               if (kFp8) {
                 const uint32_t sfid = static_cast<uint32_t>(kk) << 30;
                 mma_mxf8(d, ad + step, bd + step, idesc_mxf8(kM, nn, kk, kk, p.w_fp4 ? kFmtE2M1 : kFmtE4M3),
-                         (tbase + kSfaCol) | sfid, (tbase + kSfbCol) | sfid, acc);
+                         (tbase + sfa_col(s)) | sfid, (tbase + sfb_col(s)) | sfid, acc);
               } else {
                 mma_f16(d, ad + step, bd + step, idesc_bf16(kM, nn), acc);
               }
@@ -879,49 +937,44 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     uint4* stg4 = reinterpret_cast<uint4*>(ctrl + kP2Ctrl) + (warp - kP2FirstEpi) * (kStageFloatsPerWarp / 4);
     int acc_it = 0;
     bool ok = true;
-    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_units, n_ht, p.bm);
-    for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-      const int ht = u - (u / n_ht) * n_ht;
+    BlockPf pf = block_prefetch(p.sorted_ids, p.expert_ids, blockIdx.x, n_items, per_block, p.bm);
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      const int u = w / S2, s2 = w - u * S2, ht = u - (u / n_ht) * n_ht;
       const BlockPf cur = pf;
-      pf = block_prefetch(p.sorted_ids, p.expert_ids, u + gridDim.x, n_units, n_ht, p.bm);
+      pf = block_prefetch(p.sorted_ids, p.expert_ids, w + gridDim.x, n_items, per_block, p.bm);
       const BlockInfo bi = block_finalize(cur, p.R, p.E);
       if (bi.nend == 0) continue;
       const int nn = min(TH, p.K - ht * TH);
-      // the route and its weight, fetched while the MMAs run
+      // the route, its partial row (one per route and split of N/2) and its
+      // weight, fetched while the MMAs run
       const bool mine = row_valid(bi, r);
-      int route = 0;
+      int route = 0, prow = 0;
       float wgt = 0.f;
       if (mine) {
         route = pf_id(cur, q);
+        prow = route * S2 + s2;
         wgt = __ldg(p.topk_w + route);
       }
       const int buf = acc_it % kNumAcc;
       const uint32_t acc_ph = static_cast<uint32_t>(acc_it / kNumAcc) & 1u;
-      ok = mbar_wait(&acc_full[buf], acc_ph, abort_flag, p.status);
+      ok = mbar_wait(&acc_full[buf], acc_ph, abort_flag, p.status, p.wait_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 256u;
       bool released = false;
       if (32 * q < bi.nend && kFp8) {
-        // One TMEM accumulator on this path: the thread's weighted half-row is
-        // packed to bf16 in registers (up to 4 slices of 32 features) and the
+        // One TMEM accumulator on this path: the thread's weighted half-row
+        // (up to 4 slices of 32 fp32 features) is read into registers and the
         // accumulator handed back to the MMA warp before the slices go through
         // the staging buffer to global memory, as below.
         const int half = nn / 2;
         const int64_t col_base = static_cast<int64_t>(ht) * TH + h * half;
-        uint32_t pk[4][16];
+        uint32_t yv[4][32];
 #pragma unroll
-        for (int sl = 0; sl < 4; ++sl) {
-          if (32 * sl < half) {  // uniform
-            uint32_t yr[32];
-            tmem_ld32(tacc + h * half + 32 * sl, yr);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[sl][i] = pack_bf16x2(wgt * __uint_as_float(yr[2 * i]), wgt * __uint_as_float(yr[2 * i + 1]));
-          }
-        }
+        for (int sl = 0; sl < 4; ++sl)
+          if (32 * sl < half) tmem_ld32(tacc + h * half + 32 * sl, yv[sl]);  // uniform
+        tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -929,35 +982,42 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl) {
           if (32 * sl < half) {
-            __syncwarp();
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              stg4[lane * 4 + (i ^ ((lane >> 1) & 3))] =
-                  make_uint4(pk[sl][4 * i], pk[sl][4 * i + 1], pk[sl][4 * i + 2], pk[sl][4 * i + 3]);
-            __syncwarp();
+            for (int hh = 0; hh < 2; ++hh) {
+              __syncwarp();
 #pragma unroll
-            for (int it = 0; it < 4; ++it) {
-              const int rl = 8 * it + (lane >> 2), cq = lane & 3;
-              const uint4 v = stg4[rl * 4 + (cq ^ ((rl >> 1) & 3))];
-              const int route_l = __shfl_sync(0xffffffffu, route, rl);
-              const int mine_l = __shfl_sync(0xffffffffu, static_cast<int>(mine), rl);
-              if (mine_l) {
-                const int64_t e0 = static_cast<int64_t>(route_l) * p.K + col_base + 32 * sl;
-                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.yw) + e0 + 8 * cq) = v;
+              for (int i = 0; i < 4; ++i) {
+                const int k = 16 * hh + 4 * i;
+                stg4[lane * 4 + (i ^ ((lane >> 1) & 3))] =
+                    make_uint4(__float_as_uint(wgt * __uint_as_float(yv[sl][k])),
+                               __float_as_uint(wgt * __uint_as_float(yv[sl][k + 1])),
+                               __float_as_uint(wgt * __uint_as_float(yv[sl][k + 2])),
+                               __float_as_uint(wgt * __uint_as_float(yv[sl][k + 3])));
+              }
+              __syncwarp();
+#pragma unroll
+              for (int it = 0; it < 4; ++it) {
+                const int rl = 8 * it + (lane >> 2), cq = lane & 3;
+                const uint4 v = stg4[rl * 4 + (cq ^ ((rl >> 1) & 3))];
+                const int route_l = __shfl_sync(0xffffffffu, prow, rl);
+                const int mine_l = __shfl_sync(0xffffffffu, static_cast<int>(mine), rl);
+                if (mine_l) {
+                  const int64_t e0 = static_cast<int64_t>(route_l) * p.K + col_base + 32 * sl + 16 * hh;
+                  *reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.yw) + e0 + 4 * cq) = v;
+                }
               }
             }
           }
         }
-        if (mine && ht == 0 && h == 0) p.flags[route] = 1;
+        if (mine && ht == 0 && h == 0 && s2 == 0) p.flags[route] = 1;
       } else if (32 * q < bi.nend) {
         // Thread = row.  Each slice of the warp's 32 rows goes through shared
         // memory so that the stores leave as 64 contiguous bytes per row (8
         // rows per instruction) instead of 16 bytes to 32 different rows.
         // 16-byte slot i of row l sits at i ^ ((l >> 1) & 3), so both the
         // row-per-lane writes and the 8-rows-per-instruction reads touch all
-        // 32 banks (4 wavefronts per 512 bytes).  The bf16 path keeps the
-        // weighted rows in fp32 (16 columns per slice); the mxfp8 path rounds
-        // them to bf16 (32 columns per slice), half the bytes.
+        // 32 banks (4 wavefronts per 512 bytes).  The weighted rows stay fp32
+        // (16 columns per staging pass).
         const int half = nn / 2;
         const int64_t col_base = static_cast<int64_t>(ht) * TH + h * half;
 #pragma unroll 1
@@ -966,44 +1026,32 @@ __global__ void __launch_bounds__(kP2Threads, 1)
           tmem_ld32(tacc + h * half + c, yr);
           tmem_ld_wait();
 #pragma unroll
-          for (int hh = 0; hh < (kFp8 ? 1 : 2); ++hh) {
+          for (int hh = 0; hh < 2; ++hh) {
             __syncwarp();
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              uint4 w;
-              if (kFp8) {
-                const int k = 8 * i;
-                w = make_uint4(pack_bf16x2(wgt * __uint_as_float(yr[k]), wgt * __uint_as_float(yr[k + 1])),
-                               pack_bf16x2(wgt * __uint_as_float(yr[k + 2]), wgt * __uint_as_float(yr[k + 3])),
-                               pack_bf16x2(wgt * __uint_as_float(yr[k + 4]), wgt * __uint_as_float(yr[k + 5])),
-                               pack_bf16x2(wgt * __uint_as_float(yr[k + 6]), wgt * __uint_as_float(yr[k + 7])));
-              } else {
-                const int k = 16 * hh + 4 * i;
-                w = make_uint4(__float_as_uint(wgt * __uint_as_float(yr[k])),
-                               __float_as_uint(wgt * __uint_as_float(yr[k + 1])),
-                               __float_as_uint(wgt * __uint_as_float(yr[k + 2])),
-                               __float_as_uint(wgt * __uint_as_float(yr[k + 3])));
-              }
-              stg4[lane * 4 + (i ^ ((lane >> 1) & 3))] = w;
+              const int k = 16 * hh + 4 * i;
+              stg4[lane * 4 + (i ^ ((lane >> 1) & 3))] =
+                  make_uint4(__float_as_uint(wgt * __uint_as_float(yr[k])),
+                             __float_as_uint(wgt * __uint_as_float(yr[k + 1])),
+                             __float_as_uint(wgt * __uint_as_float(yr[k + 2])),
+                             __float_as_uint(wgt * __uint_as_float(yr[k + 3])));
             }
             __syncwarp();
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
               const int rl = 8 * it + (lane >> 2), cq = lane & 3;
               const uint4 v = stg4[rl * 4 + (cq ^ ((rl >> 1) & 3))];
-              const int route_l = __shfl_sync(0xffffffffu, route, rl);
+              const int route_l = __shfl_sync(0xffffffffu, prow, rl);
               const int mine_l = __shfl_sync(0xffffffffu, static_cast<int>(mine), rl);
               if (mine_l) {
                 const int64_t e0 = static_cast<int64_t>(route_l) * p.K + col_base + c;
-                if (kFp8)
-                  *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.yw) + e0 + 8 * cq) = v;
-                else
-                  *reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.yw) + e0 + 16 * hh + 4 * cq) = v;
+                *reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.yw) + e0 + 16 * hh + 4 * cq) = v;
               }
             }
           }
         }
-        if (mine && ht == 0 && h == 0) p.flags[route] = 1;
+        if (mine && ht == 0 && h == 0 && s2 == 0) p.flags[route] = 1;
       }
       if (!released) {
         tc_fence_before();
@@ -1024,50 +1072,19 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 }
 
 // ========================================================================
-// combine: out[t] = bf16( sum_j yw[t*top_k + j] ), routes in order
+// combine: out[t] = bf16( sum over j, s of yw[(t*top_k + j)*nsplit2 + s] ),
+// routes in order
 // ========================================================================
-// 8 consecutive partials of one route, kept packed in registers until they
-// are summed (bf16: one 16-byte load, fp32: two), so that a thread holds all
-// of its routes' loads in flight with few registers.
-template <typename TP>
-struct Raw8;
-template <>
-struct Raw8<__nv_bfloat16> {
-  uint4 a;
-};
-template <>
-struct Raw8<float> {
-  uint4 a, b;
-};
-__device__ __forceinline__ void load_raw8(const __nv_bfloat16* p, Raw8<__nv_bfloat16>& r) {
-  r.a = __ldg(reinterpret_cast<const uint4*>(p));
-}
-__device__ __forceinline__ void load_raw8(const float* p, Raw8<float>& r) {
-  r.a = __ldg(reinterpret_cast<const uint4*>(p));
-  r.b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
-}
-__device__ __forceinline__ void add_raw8(const Raw8<__nv_bfloat16>& r, float (&acc)[8]) {
-  const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc[2 * i] += __uint_as_float(w[i] << 16);
-    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-__device__ __forceinline__ void add_raw8(const Raw8<float>& r, float (&acc)[8]) {
-  const uint32_t w[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] += __uint_as_float(w[i]);
-}
-
 // One thread sums 8 consecutive features of one token over its top_k routes.
 // The route flags and every route's 8 partials are loaded before any of them
 // is used (the loads of a route whose flag is 0 read workspace bytes that are
 // then discarded), so a thread has all its loads in flight at once; the sum
 // runs in route order, so the result does not depend on scheduling.
-template <typename TP, int kMaxK>
-__global__ void __launch_bounds__(256, sizeof(TP) == 2 ? 4 : 2) moe_combine_kernel(const TP* __restrict__ yw, const int32_t* __restrict__ flags,
-                                                          __nv_bfloat16* __restrict__ out, int T, int K, int top_k) {
+template <int kMaxK>
+__global__ void __launch_bounds__(256, 2) moe_combine_kernel(const float* __restrict__ yw,
+                                                             const int32_t* __restrict__ flags,
+                                                             __nv_bfloat16* __restrict__ out, int T, int K,
+                                                             int top_k, int nsplit2) {
   pdl_wait();  // the down phase's partial rows are read below
   const int kv = K / 8;
   const int64_t n = static_cast<int64_t>(T) * kv;
@@ -1076,21 +1093,31 @@ __global__ void __launch_bounds__(256, sizeof(TP) == 2 ? 4 : 2) moe_combine_kern
     const int64_t t = v / kv;
     const int h = static_cast<int>(v - t * kv) * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j0 = 0; j0 < top_k; j0 += kMaxK) {
+    // the token's partial rows: route j, split s at row (t * top_k + j) * nsplit2 + s, summed in
+    // that (route-major) order
+    const int nrows = top_k * nsplit2;
+    for (int j0 = 0; j0 < nrows; j0 += kMaxK) {
       int f[kMaxK];
-      Raw8<TP> y[kMaxK];
+      uint4 y[kMaxK][2];
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j) {
         f[j] = 0;
-        if (j0 + j < top_k) {
-          const int64_t r = t * top_k + j0 + j;
-          f[j] = __ldg(flags + r);
-          load_raw8(yw + r * K + h, y[j]);
+        if (j0 + j < nrows) {
+          const int64_t r = t * nrows + j0 + j;
+          f[j] = __ldg(flags + t * top_k + (j0 + j) / nsplit2);
+          const uint4* src = reinterpret_cast<const uint4*>(yw + r * K + h);
+          y[j][0] = __ldg(src);
+          y[j][1] = __ldg(src + 1);
         }
       }
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j)
-        if (f[j]) add_raw8(y[j], acc);
+        if (f[j]) {
+          const uint32_t w[8] = {y[j][0].x, y[j][0].y, y[j][0].z, y[j][0].w,
+                                 y[j][1].x, y[j][1].y, y[j][1].z, y[j][1].w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] += __uint_as_float(w[i]);
+        }
     }
     __nv_bfloat162 o[4];
 #pragma unroll
@@ -1109,6 +1136,21 @@ struct WsLayout {
 
 static int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
+// Splits of the down GEMM's N/2 contraction: small calls (at most 64 down
+// units even if every planner block were used) spread it over up to 4 CTAs
+// per unit, each writing its own partial row, which the combine adds in
+// order.  A function of the problem's sizes only (the workspace size follows
+// from it).
+static int down_splits(bool fp8, int T, int K, int N, int E, int top_k, int bm) {
+  const int64_t R = static_cast<int64_t>(T) * top_k;
+  const int64_t blocks = round_up(R + static_cast<int64_t>(E) * (bm - 1), bm) / bm;
+  const int64_t units = blocks * ((K + kTH - 1) / kTH);
+  const int I = N / 2;
+  const int n_kc = fp8 ? I / 128 : (I + 63) / 64;
+  if (units > 64) return 1;
+  return std::max(1, std::min(4, n_kc / 2));
+}
+
 static WsLayout ws_layout(bool fp8, int T, int K, int N, int E, int top_k, int bm) {
   WsLayout w{};
   const int64_t R = static_cast<int64_t>(T) * top_k;
@@ -1121,7 +1163,7 @@ static WsLayout ws_layout(bool fp8, int T, int K, int N, int E, int top_k, int b
   w.act_sf = off;
   if (fp8) off = round_up(off + (w.cap_rows / bm) * (I / 128) * kSfTileBytes, 1024);
   w.yw = off;
-  off = round_up(off + R * K * (fp8 ? 2 : 4), 1024);
+  off = round_up(off + R * down_splits(fp8, T, K, N, E, top_k, bm) * K * 4, 1024);
   w.flags = off;
   off = round_up(off + R * 4, 1024);
   w.part = off;
@@ -1314,6 +1356,8 @@ static int run_fused(const FusedArgs& a) {
   const int nsm = sm_count();
   if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(SM count)");
   const int req_stages = a.tune ? a.tune->stages : 0;
+  const unsigned long long wait_ns =
+      a.tune && a.tune->wait_timeout_ns > 0 ? static_cast<unsigned long long>(a.tune->wait_timeout_ns) : kWaitTimeoutNs;
   const int req_ctas = a.tune ? a.tune->num_ctas : 0;
   // Blocks a kernel may visit: never past the caller's sorted_token_ids /
   // expert_ids arrays, even if num_tokens_post_padded were out of range.
@@ -1340,7 +1384,25 @@ static int run_fused(const FusedArgs& a) {
   p1.stage_bytes = stage_bytes(a.fp8, a_rows);
   p1.off_b = off_b_of(a_rows);
   p1.off_sf = off_sf_of(a_rows);
-  p1.stages = pick_stages(p1.stage_bytes, kP1Ctrl, req_stages, 8);
+  p1.stages = pick_stages(p1.stage_bytes, kP1Ctrl, req_stages, kMaxStages);
+  p1.wait_ns = wait_ns;
+  {
+    // L2 prefetch (see P1Params): the whole expert set when it is small, else
+    // the down phase's touched w2 tiles when they are
+    const int64_t wb1 = static_cast<int64_t>(a.E) * a.N * a.K * (a.fp8 ? 1 : 2) / (a.w_fp4 ? 2 : 1);
+    const int64_t wb2 = static_cast<int64_t>(a.E) * a.K * I * (a.fp8 ? 1 : 2) / (a.w_fp4 ? 2 : 1);
+    const int64_t sb1 = a.fp8 ? pack_scales_blocked_bytes(a.E, a.N, a.K / 32) : 0;
+    const int64_t sb2 = a.fp8 ? pack_scales_blocked_bytes(a.E, a.K, I / 32) : 0;
+    p1.pf_all = wb1 + wb2 + sb1 + sb2 <= kPrefetchAllBytes ? 1 : 0;
+    p1.pf_src[0] = static_cast<const uint8_t*>(a.w1); p1.pf_bytes[0] = wb1;
+    p1.pf_src[1] = static_cast<const uint8_t*>(a.w2); p1.pf_bytes[1] = wb2;
+    p1.pf_src[2] = a.w1_sf; p1.pf_bytes[2] = a.w1_sf ? sb1 : 0;
+    p1.pf_src[3] = a.w2_sf; p1.pf_bytes[3] = a.w2_sf ? sb2 : 0;
+    p1.w2 = static_cast<const uint8_t*>(a.w2);
+    p1.w2_sf = a.fp8 ? a.w2_sf : nullptr;
+    p1.w2_row_bytes = static_cast<int64_t>(I) * (a.fp8 ? 1 : 2) / (a.w_fp4 ? 2 : 1);
+    p1.pf_w2_budget = kPrefetchW2Bytes;
+  }
 
   P2Params p2{};
   p2.w2_sf = a.w2_sf;
@@ -1358,15 +1420,17 @@ static int run_fused(const FusedArgs& a) {
   p2.w_fp4 = p1.w_fp4;
   p2.n_ht = (a.K + kTH - 1) / kTH;
   p2.n_kc = a.fp8 ? I / 128 : (I + 63) / 64;
+  p2.nsplit2 = down_splits(a.fp8, a.T, a.K, a.N, a.E, a.top_k, a.bm);
   p2.stage_bytes = stage_bytes(a.fp8, a_rows);
   p2.off_b = p1.off_b;
   p2.a_full = a_rows >= kM ? 1 : 0;
   p2.off_sf = p1.off_sf;
-  p2.stages = pick_stages(p2.stage_bytes, kP2Ctrl + kP2Staging, req_stages, 8);
+  p2.stages = pick_stages(p2.stage_bytes, kP2Ctrl + kP2Staging, req_stages, kMaxStages);
+  p2.wait_ns = wait_ns;
   if (p1.stages < 2 || p2.stages < 2) return fail(MOE_ERR_UNSUPPORTED, "%s: shared memory too small", nm);
 
   const int64_t units1 = static_cast<int64_t>(max_blocks) * p1.n_jt;
-  const int64_t units2 = static_cast<int64_t>(max_blocks) * p2.n_ht;
+  const int64_t units2 = static_cast<int64_t>(max_blocks) * p2.n_ht * p2.nsplit2;
   int ctas = req_ctas > 0 ? req_ctas : nsm;
   // one CTA per SM: small problems split their units' K range over the CTAs
   const int grid1 = ctas;
@@ -1424,27 +1488,23 @@ static int run_fused(const FusedArgs& a) {
   if (err != cudaSuccess) return cuda_fail("fused_moe: down phase launch", err);
   if ((rc = mark(2)) != MOE_OK) return rc;
   // one full wave of resident blocks (grid-stride beyond it)
-  static std::atomic<int> comb_occ[2];  // races store the same value
-  int occ = comb_occ[a.fp8 ? 1 : 0].load(std::memory_order_relaxed);
+  static std::atomic<int> comb_occ;  // races store the same value
+  int occ = comb_occ.load(std::memory_order_relaxed);
   if (occ == 0) {
     int nb = 0;
-    err = a.fp8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<__nv_bfloat16, 8>, 256, 0)
-                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<float, 8>, 256, 0);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<8>, 256, 0);
     if (err != cudaSuccess) return cuda_fail("fused_moe: combine occupancy query", err);
     occ = nb < 1 ? 1 : nb;
-    comb_occ[a.fp8 ? 1 : 0].store(occ, std::memory_order_relaxed);
+    comb_occ.store(occ, std::memory_order_relaxed);
   }
   const int64_t nvec = static_cast<int64_t>(a.T) * (a.K / 8);
   const int64_t cblocks = (nvec + 255) / 256;
   const int64_t wave = static_cast<int64_t>(occ) * nsm;
   const int cgrid = static_cast<int>(cblocks < wave ? cblocks : wave);
   cudaLaunchConfig_t c3 = config(cgrid, 256, 0);
-  __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(a.out);
-  err = a.fp8 ? cudaLaunchKernelEx(&c3, moe_combine_kernel<__nv_bfloat16, 8>,
-                                   reinterpret_cast<const __nv_bfloat16*>(ws + L.yw),
-                                   static_cast<const int32_t*>(p1.flags), outp, a.T, a.K, a.top_k)
-              : cudaLaunchKernelEx(&c3, moe_combine_kernel<float, 8>, reinterpret_cast<const float*>(ws + L.yw),
-                                   static_cast<const int32_t*>(p1.flags), outp, a.T, a.K, a.top_k);
+  err = cudaLaunchKernelEx(&c3, moe_combine_kernel<8>, reinterpret_cast<const float*>(ws + L.yw),
+                           static_cast<const int32_t*>(p1.flags), static_cast<__nv_bfloat16*>(a.out), a.T, a.K,
+                           a.top_k, p2.nsplit2);
   if (err != cudaSuccess) return cuda_fail("fused_moe: combine launch", err);
   return mark(3);
 }

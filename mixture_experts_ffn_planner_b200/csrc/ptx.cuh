@@ -61,18 +61,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits until the phase with the given parity has completed.  Gives up (and
-// returns false) when the CTA-wide abort flag is raised or after
-// kWaitTimeoutNs; a timeout raises the abort flag and records
-// MOE_ERR_TIMEOUT (-6) in the device status word *status.
+// returns false) when the CTA-wide abort flag is raised or after limit_ns
+// (kWaitTimeoutNs unless the caller set a test limit); a timeout raises the
+// abort flag and records MOE_ERR_TIMEOUT (-6) in the device status word
+// *status.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
+  // the timer is read every 16 polls, or on every poll under a short (test) limit
+  const uint32_t mask = limit_ns < 1000000ull ? 0u : 15u;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 15u) == 0) {
+    if ((it & mask) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitTimeoutNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicExch(status, -6);
         return false;
@@ -102,6 +105,14 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// Prefetches [src, src + bytes) of global memory into L2 (no shared memory
+// involved, no completion to wait for); src 16-byte aligned, bytes a
+// multiple of 16.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
 }
 
 // 2-D tiled TMA load (no multicast): box at (c0 = inner element, c1 = row).

@@ -6,17 +6,20 @@ mxfp8 path (the oracle emulates the on-chip requant): cosine >= 0.999 and
 max|gpu - oracle| <= 6e-2 * rms(oracle out).  "oracle out" is the oracle's
 result before its final rounding to bf16 (see tests/helpers.py).
 Small cases run the whole oracle; they span several 128-row blocks, several
-intermediate tiles and a ragged tail.  The named workloads at full size are
-checked on a seeded token sample that always includes tokens of the most-
-and least-loaded experts (tokens are independent, so their rows are exact
-sub-results).
+intermediate tiles and a ragged tail.  The named workloads at full size run
+the whole oracle up to 256 tokens and otherwise a seeded sample of 512 tokens
+(tokens are independent, so their rows are exact sub-results) that covers
+every non-empty expert, the last row of full blocks and the last block
+(tests/helpers.coverage_sample).
 """
 import numpy as np
 import pytest
 
 import oracle
 import workloads as W
-from tests.helpers import assert_bf16_parity, assert_mxfp8_parity, out_bits, to_dev
+from tests.helpers import assert_bf16_parity, assert_mxfp8_parity, coverage_sample, out_bits, to_dev
+
+FULL_SAMPLE = 512  # tokens compared at full size (the whole batch when it is smaller)
 
 pytestmark = pytest.mark.gpu
 
@@ -148,11 +151,12 @@ def test_c1_full():
 
 
 @pytest.mark.parametrize("T", [1, 8, 64, 512, 8192])
-def test_c5_sampled(T):
-    """bf16 narrow intermediate with Zipf-skewed routing (empty experts)."""
+def test_c5(T):
+    """bf16 narrow intermediate with Zipf-skewed routing (empty experts): whole batch up to T=512,
+    a 512-token coverage sample at T=8192."""
     sh = W.shape("C5", T)
     inp = W.inputs(sh)
-    toks = W.sample_tokens(sh, inp["topk_ids"], 48)
+    toks = coverage_sample(sh, inp["topk_ids"], FULL_SAMPLE)
     got = gpu_forward(sh, inp)
     ref = oracle_forward(sh, inp, tokens=toks)
     rel, cos = check(sh, got[toks], ref[toks], f"C5 T={T}")
@@ -189,19 +193,22 @@ def _full_inputs(name, T):
     return sh, inp
 
 
-@pytest.mark.parametrize("name,T,ntok", [("C2", 64, 32), ("C2", 256, 32),
-                                         ("C3", 64, 12), ("C3", 256, 12), ("C3", 1024, 12), ("C3", 2048, 12),
-                                         ("C3", 4096, 12), ("C3", 8192, 12),
-                                         ("C4", 1024, 6), ("C4", 2048, 6), ("C4", 4096, 6), ("C4", 8192, 6),
-                                         ("C3F4", 64, 12), ("C3F4", 2048, 12), ("C3F4", 8192, 12),
-                                         ("C4F4", 1024, 6), ("C4F4", 8192, 6)])
-def test_full_size_sampled(name, T, ntok):
-    """The workload at full size through the GPU path; parity on a seeded token
-    sample that includes tokens of the most- and least-loaded experts."""
+FULL_CASES = [("C2", 64), ("C2", 256),
+              ("C3", 64), ("C3", 256), ("C3", 1024), ("C3", 2048), ("C3", 4096), ("C3", 8192),
+              ("C4", 1024), ("C4", 2048), ("C4", 4096), ("C4", 8192),
+              ("C3F4", 64), ("C3F4", 2048), ("C3F4", 8192),
+              ("C4F4", 1024), ("C4F4", 8192)]
+
+
+@pytest.mark.parametrize("name,T", FULL_CASES)
+def test_full_size(name, T):
+    """The workload at full size through the GPU path; parity on the whole batch (T <= 256) or a
+    512-token coverage sample (every non-empty expert, block tails, the last block)."""
     sh, inp = _full_inputs(name, T)
-    toks = W.sample_tokens(sh, inp["topk_ids"], ntok)
+    toks = coverage_sample(sh, inp["topk_ids"], FULL_SAMPLE)
     got = gpu_forward(sh, inp)
     ref = oracle_forward(sh, inp, tokens=toks)
     rel, cos = check(sh, got[toks], ref[toks], f"{name} T={T}")
     assert np.isfinite(W.bf16_bits_to_f32(got)).all()
-    print(f"PARITY {name} T={T} tokens={len(toks)} max|diff|/rms={rel:.3e} cos={cos:.7f}")
+    print(f"PARITY {name} T={T} tokens={len(toks)} experts={len(np.unique(inp['topk_ids'][toks]))} "
+          f"max|diff|/rms={rel:.3e} cos={cos:.7f}")

@@ -129,21 +129,26 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 
 
 def mx_quantize_inputs(v: np.ndarray):
-    """Caller-side OCP MX quantiser: (..., L) fp32 -> e4m3 codes (..., L), e8m0 (..., L/32)."""
+    """Caller-side OCP MX quantiser: (..., L) fp32 -> e4m3 codes (..., L), e8m0 (..., L/32).
+
+    Scale 2^(floor(log2 amax) - 8) per block of 32 (8 = emax of e4m3; an all-zero block gets byte
+    0), values multiplied by the inverse power of two in fp32, clamped to +-448 and rounded to e4m3
+    by torch's float8_e4m3fn conversion (round to nearest even).  The elementwise passes run as
+    torch CPU ops (multi-threaded); the per-block scale arithmetic in numpy."""
     import torch
 
     v = np.ascontiguousarray(v, dtype=np.float32)
     L = v.shape[-1]
     assert L % 32 == 0
-    blk = v.reshape(-1, 32)
-    amax = np.abs(blk).max(axis=1)
+    blk = torch.from_numpy(v).view(-1, 32)
+    amax = blk.abs().amax(dim=1).numpy()
     _, ex = np.frexp(amax)                      # amax = m * 2^ex, 0.5 <= m < 1
     shared = ex.astype(np.int32) - 1 - 8        # floor(log2 amax) - emax(e4m3)
     shared = np.where(amax > 0, shared, -127)
     shared = np.clip(shared, -127, 127)
-    mult = np.ldexp(np.float32(1.0), (-shared).astype(np.int32)).astype(np.float32)
-    scaled = np.clip(blk * mult[:, None], -448.0, 448.0).astype(np.float32)
-    codes = torch.from_numpy(scaled).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mult = torch.from_numpy(np.ldexp(np.float32(1.0), (-shared).astype(np.int32)).astype(np.float32))
+    scaled = (blk * mult[:, None]).clamp_(-448.0, 448.0)
+    codes = scaled.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     return codes.reshape(v.shape), (shared + 127).astype(np.uint8).reshape(v.shape[:-1] + (L // 32,))
 
 
@@ -229,35 +234,29 @@ def bf16_inputs(sh: Shape, seed: int = DEFAULT_SEED, threads: int | None = None)
                 w2=bf16_weights(sh, "w2", seed, threads), topk_ids=ids, topk_weights=tw)
 
 
-# OCP E2M1 magnitudes by 3-bit code (exponent bias 1, one mantissa bit)
-_E2M1_MAG = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0], dtype=np.float64)
-
-
 def mx_quantize_fp4(v: np.ndarray):
     """Caller-side OCP MX FP4 quantiser: (..., L) fp32 -> packed e2m1 codes (..., L/2) u8 (value
     2j in the low nibble of byte j) and e8m0 scales (..., L/32).  Shared scale
-    2^(floor(log2 amax) - 2) (emax of e2m1 is 2); values rounded to the nearest e2m1 magnitude,
-    ties to the even code, beyond 6 saturated; an all-zero block gets scale byte 0."""
+    2^(floor(log2 amax) - 2) (emax of e2m1 is 2); values rounded to the nearest e2m1 magnitude
+    (0, 0.5, 1, 1.5, 2, 3, 4, 6), ties to the even code, beyond 6 saturated; an all-zero block gets
+    scale byte 0.  The code of a scaled magnitude m is the number of rounding boundaries it has
+    passed: 0.25, 1.25, 2.5 and 5 round down on a tie (the lower code is even), 0.75, 1.75 and 3.5
+    round up; the sign bit is 8.  Elementwise passes as torch CPU ops in float64 (exact)."""
+    import torch
+
     v = np.ascontiguousarray(v, dtype=np.float32)
     L = v.shape[-1]
     assert L % 32 == 0
-    blk = v.reshape(-1, 32).astype(np.float64)
-    amax = np.abs(blk).max(axis=1)
+    blk = torch.from_numpy(v).view(-1, 32).double()
+    amax = blk.abs().amax(dim=1).numpy()
     _, ex = np.frexp(amax)
     shared = np.where(amax > 0, ex.astype(np.int32) - 1 - 2, -127)
     shared = np.clip(shared, -127, 127)
-    scaled = blk * np.ldexp(1.0, -shared)[:, None]
-    mag = np.abs(scaled)
-    # nearest magnitude by exhaustive comparison; on a tie the even code (smaller index with
-    # an even mantissa bit) wins
-    d = np.abs(mag[..., None] - _E2M1_MAG[None, None, :])
-    best = np.argmin(d, axis=-1)
-    dmin = np.take_along_axis(d, best[..., None], axis=-1)[..., 0]
-    nxt = np.minimum(best + 1, 7)
-    tie = (np.take_along_axis(d, nxt[..., None], axis=-1)[..., 0] == dmin) & (nxt != best)
-    best = np.where(tie & (best % 2 == 1), nxt, best)
-    best = np.where(mag >= 6.0, 7, best)
-    codes = (best | np.where(np.signbit(scaled), 8, 0)).astype(np.uint8).reshape(v.shape)
+    scaled = blk * torch.from_numpy(np.ldexp(1.0, -shared))[:, None]
+    mag = scaled.abs()
+    code = ((mag > 0.25).to(torch.uint8) + (mag >= 0.75) + (mag > 1.25) + (mag >= 1.75) + (mag > 2.5)
+            + (mag >= 3.5) + (mag > 5.0))
+    codes = (code | (torch.signbit(scaled).to(torch.uint8) << 3)).numpy().reshape(v.shape)
     packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
     scales = (shared + 127).astype(np.uint8).reshape(v.shape[:-1] + (L // 32,))
     return packed, scales
