@@ -251,6 +251,42 @@ MOE_API int fused_moe_mxfp4(const uint8_t* x_e4m3, const uint8_t* x_scales, cons
                     const moe_tuning* tune, moe_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Expert-parallel dispatch and combine -- DeepGEMM #411 "SM90 FP8 x MXFP4
+ * MegaMoE", Summary, and "[SM90] Ring-buffered FP8 MegaMoE with a lag-ordered
+ * L1/L2 schedule" (sgl DeepGEMM PR #88): the experts are sharded over the
+ * `world` ranks of a group (rank r owns experts [r*E/world, (r+1)*E/world)),
+ * each routed row goes to the owner of its expert (dispatch), the owners run
+ * their experts, and the results come back to be summed per token (combine).
+ * The exchanges are the caller's collectives; these calls do the device work
+ * on either side.  All pointers device, caller-owned; asynchronous on
+ * `stream`.  Constraints: 1 <= world <= 64, E % world == 0.
+ *
+ * moe_ep_dispatch_plan -- order (T*top_k int32, written in full): the route
+ *   ids t*top_k+j whose expert is in [0, E), grouped by owner rank (rank 0
+ *   first), ascending inside a group, then -1; send_counts (world int32): the
+ *   size of each group.
+ * moe_ep_dispatch_pack -- for i < n (n = sum of send_counts): rows_out[i] =
+ *   the row (row_bytes bytes) of x of token order[i] / top_k; scales_out[i] =
+ *   its scale row (scale_bytes bytes) when x_scales is not NULL;
+ *   local_expert_out[i] = its expert minus the owner's first expert;
+ *   weight_out[i] = its routing weight.  x and rows_out 16-byte aligned when
+ *   row_bytes % 16 == 0.
+ * moe_ep_combine -- y (n, K) bf16: the returned rows, row i for route
+ *   order[i]; slot: T*top_k int32 scratch; out (T, K) bf16, overwritten:
+ *   out[t] = bf16( sum over j of y[row of route t*top_k+j] ), routes in order,
+ *   fp32 sums; a token none of whose routes is in `order` gets zeros.  K % 8
+ *   == 0; y and out 16-byte aligned.
+ * ---------------------------------------------------------------------- */
+MOE_API int moe_ep_dispatch_plan(const int32_t* topk_ids, int T, int top_k, int E, int world, int32_t* order,
+                                 int32_t* send_counts, moe_stream_t stream);
+MOE_API int moe_ep_dispatch_pack(const void* x, int64_t row_bytes, const uint8_t* x_scales, int64_t scale_bytes,
+                                 const int32_t* topk_ids, const float* topk_weights, const int32_t* order, int n,
+                                 int T, int top_k, int E, int world, void* rows_out, uint8_t* scales_out,
+                                 int32_t* local_expert_out, float* weight_out, moe_stream_t stream);
+MOE_API int moe_ep_combine(const void* y, const int32_t* order, int n, int T, int top_k, int K, int32_t* slot,
+                           void* out, moe_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * fused_moe_bf16_noalloc -- the pages have no counterpart to this call; it
  * is a convenience of this library.  It computes exactly what
  * fused_moe_bf16 computes, for callers that cannot allocate device memory

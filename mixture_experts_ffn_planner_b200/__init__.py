@@ -22,6 +22,9 @@ Entry points (same names as the C ABI):
   values per byte (DeepGEMM #411 "SM90 FP8 x MXFP4 MegaMoE" operand pairing).
 * ``pack_scales_blocked`` -- weight scales into 512-byte tiles of
   128 MN x 128 K ("Prime Flash MoE", Scale layout (mxfp8)).
+* ``moe_ep_dispatch_plan`` / ``moe_ep_dispatch_pack`` / ``moe_ep_combine`` --
+  the device work around an expert-parallel exchange (DeepGEMM #411 "SM90 FP8
+  x MXFP4 MegaMoE", Summary: dispatch, routed experts, combine).
 """
 from __future__ import annotations
 
@@ -37,7 +40,7 @@ __all__ = [
     "fused_moe_mxfp4", "DTYPE_MXFP4",
     "pack_scales_blocked", "pack_scales_blocked_bytes", "moe_workspace_bytes", "moe_device_status",
     "Tuning", "DTYPE_BF16", "DTYPE_MXFP8", "LIB_PATH", "fused_moe_bf16_noalloc",
-    "fused_moe_bf16_noalloc_max_workspace",
+    "fused_moe_bf16_noalloc_max_workspace", "moe_ep_dispatch_plan", "moe_ep_dispatch_pack", "moe_ep_combine",
 ]
 
 DTYPE_BF16 = 0
@@ -96,6 +99,9 @@ _SIGS = {
     "fused_moe_mxfp4": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _I64,
                          _P, _P], _I),
     "fused_moe_bf16_noalloc_max_workspace": ([], _I64),
+    "moe_ep_dispatch_plan": ([_P, _I, _I, _I, _I, _P, _P, _P], _I),
+    "moe_ep_dispatch_pack": ([_P, _I64, _P, _I64, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P], _I),
+    "moe_ep_combine": ([_P, _P, _I, _I, _I, _I, _P, _P, _P], _I),
     "fused_moe_bf16_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _P, _P], _I),
 }
 
@@ -455,6 +461,80 @@ def fused_moe_bf16_noalloc(x, w1, w2, sorted_token_ids, expert_ids, num_tokens_p
             _ptr(x), _ptr(w1), _ptr(w2), _ptr(sorted_token_ids), _ptr(expert_ids), _ptr(num_tokens_post_padded),
             _ptr(topk_weights), _ptr(out), T, K, N, E, top_k, block_m, sorted_token_ids.numel(),
             None if tune is None else ctypes.byref(tune), s))
+    return out
+
+
+def moe_ep_dispatch_plan(topk_ids, E: int, world: int, order=None, send_counts=None, stream=None):
+    """Routes grouped by owner rank (experts split into `world` equal ranges).  Returns (order
+    (T*top_k,) int32: route ids t*top_k+j reaching an expert, grouped by rank, then -1;
+    send_counts (world,) int32)."""
+    import torch
+
+    _need(topk_ids, "topk_ids", (torch.int32,))
+    T, top_k = topk_ids.shape
+    dev = topk_ids.device
+    order = torch.empty(T * top_k, dtype=torch.int32, device=dev) if order is None else order
+    send_counts = torch.empty(world, dtype=torch.int32, device=dev) if send_counts is None else send_counts
+    _need(order, "order", (torch.int32,))
+    _need(send_counts, "send_counts", (torch.int32,))
+    if order.numel() < T * top_k or send_counts.numel() < world:
+        raise ValueError("order must hold T*top_k entries and send_counts world entries")
+    _same_device(topk_ids, order, send_counts)
+    with _on_device(dev, stream) as s:
+        _check(load().moe_ep_dispatch_plan(_ptr(topk_ids), T, top_k, E, world, _ptr(order), _ptr(send_counts), s))
+    return order, send_counts
+
+
+def moe_ep_dispatch_pack(x, topk_ids, topk_weights, order, n: int, E: int, world: int, x_scales=None, stream=None):
+    """The send buffers of the first n entries of `order`: (rows (n, K) in x's dtype, scales (n, K/32) uint8 or
+    None, owner-local expert ids (n,) int32, routing weights (n,) fp32)."""
+    import torch
+
+    _need(topk_ids, "topk_ids", (torch.int32,))
+    _need(topk_weights, "topk_weights", (torch.float32,))
+    _need(order, "order", (torch.int32,))
+    if not x.is_contiguous() or x.dim() != 2:
+        raise ValueError("x must be a contiguous (T, K) tensor")
+    T, top_k = topk_ids.shape
+    if x.shape[0] != T or tuple(topk_weights.shape) != (T, top_k) or order.numel() < n:
+        raise ValueError("x, topk_ids, topk_weights and order disagree in shape")
+    dev = x.device
+    rows = torch.empty((n, x.shape[1]), dtype=x.dtype, device=dev)
+    scales = None
+    if x_scales is not None:
+        _need(x_scales, "x_scales", (torch.uint8,))
+        if x_scales.shape[0] != T:
+            raise ValueError("x_scales must have one row per token")
+        scales = torch.empty((n, x_scales.shape[1]), dtype=torch.uint8, device=dev)
+    local_e = torch.empty(n, dtype=torch.int32, device=dev)
+    w = torch.empty(n, dtype=torch.float32, device=dev)
+    _same_device(x, topk_ids, topk_weights, order, *([] if x_scales is None else [x_scales]))
+    with _on_device(dev, stream) as s:
+        _check(load().moe_ep_dispatch_pack(
+            _ptr(x), x.shape[1] * x.element_size(), _ptr(x_scales), 0 if x_scales is None else x_scales.shape[1],
+            _ptr(topk_ids), _ptr(topk_weights), _ptr(order), n, T, top_k, E, world, _ptr(rows), _ptr(scales),
+            _ptr(local_e), _ptr(w), s))
+    return rows, scales, local_e, w
+
+
+def moe_ep_combine(y, order, n: int, T: int, top_k: int, out=None, slot=None, stream=None):
+    """out (T, K) bf16: per token, the sum in route order (fp32) of its routes' rows of y (n, K) bf16, row i
+    belonging to route order[i]."""
+    import torch
+
+    _need(y, "y", (torch.bfloat16,))
+    _need(order, "order", (torch.int32,))
+    K = y.shape[1]
+    dev = y.device
+    out = torch.empty((T, K), dtype=torch.bfloat16, device=dev) if out is None else out
+    slot = torch.empty(max(T * top_k, 1), dtype=torch.int32, device=dev) if slot is None else slot
+    _need(out, "out", (torch.bfloat16,))
+    _need(slot, "slot", (torch.int32,))
+    if tuple(out.shape) != (T, K) or slot.numel() < T * top_k or y.shape[0] < n or order.numel() < n:
+        raise ValueError("out must be (T, K), slot hold T*top_k entries, y and order n rows")
+    _same_device(y, order, out, slot)
+    with _on_device(dev, stream) as s:
+        _check(load().moe_ep_combine(_ptr(y), _ptr(order), n, T, top_k, K, _ptr(slot), _ptr(out), s))
     return out
 
 

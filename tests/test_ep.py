@@ -6,8 +6,10 @@ combine: every rank's result must equal the single-process oracle on that rank's
 experts, in float64 to the last bit (routes are summed in the same order).  Covers routes that cross
 ranks, routes to nowhere (id -1), a rank with no tokens, and all routes landing on one rank; on the
 mxfp8 path each row's e8m0 scales travel with its e4m3 codes.
-The GPU ranks of this path (NCCL between B200s) are not exercised here: every GPU run here has one
-GPU.
+The device work on either side of the exchanges (plan, pack, combine) runs as the plain torch ops of
+tests/ep_reference_ops.py here, since CPU tensors cannot reach the kernels; the kernels are checked
+against those same ops on the GPU (tests/test_gpu_ep.py).  The GPU ranks of this path (NCCL between
+B200s) are not exercised here: every GPU run here has one GPU.
 """
 import os
 import socket
@@ -65,6 +67,7 @@ def _worker(rank, world, port, mode, results, fmt="bf16"):
     import oracle
     import workloads as W
     from mixture_experts_ffn_planner_b200.ep import ep_forward
+    from tests.ep_reference_ops import TorchOps
 
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
@@ -94,10 +97,11 @@ def _worker(rank, world, port, mode, results, fmt="bf16"):
 
         ids_t, tw_t = torch.from_numpy(ids).reshape(T, 2), torch.from_numpy(tw).reshape(T, 2)
         if fmt == "mxfp8":
-            out = ep_forward(torch.from_numpy(xq), ids_t, tw_t, E, local_ffn, x_scales=torch.from_numpy(xs))
+            out = ep_forward(torch.from_numpy(xq), ids_t, tw_t, E, local_ffn, x_scales=torch.from_numpy(xs),
+                             ops=TorchOps())
         else:
             xt = torch.from_numpy(W.bf16_bits_to_f32(x)) if T else torch.zeros((0, K), dtype=torch.float32)
-            out = ep_forward(xt, ids_t, tw_t, E, local_ffn)
+            out = ep_forward(xt, ids_t, tw_t, E, local_ffn, ops=TorchOps())
         if T:
             if fmt == "mxfp8":
                 ref = oracle.fused_moe_mxfp8(xq, xs, w1q, w1s, w2q, w2s, ids, tw, unrounded=True)[1]
