@@ -148,20 +148,21 @@ def cost_model(sh: W.Shape, topk_ids: np.ndarray, peaks: dict):
     p_tc = tensor_peak(sh, peaks) * 1e12
     bw = peaks["hbm_gbs"] * 1e9
     t_flop, t_hbm = flops / p_tc, bytes_w / bw
-    # bytes per activation value: bf16 2, mxfp8 1 + 1/32
+    # bytes per activation value: bf16 2, mxfp8 1 + 1/32; per partial-row value: fp32 / bf16
     bx = 2.0 if sh.dtype == "bf16" else 1.0 + 1.0 / 32.0
+    by = 4.0 if sh.dtype == "bf16" else 2.0
     kern = {
         # gate/up: w1 of the touched experts, the routed rows of x, the intermediate written once
         "gate_up": dict(bytes=touched * sh.N * sh.K * b + Rv * sh.K * bx + Rv * sh.I * bx,
                         flops=2.0 * Rv * sh.K * sh.N, name="moe_p1_kernel (gather + gate/up GEMM + SwiGLU)",
                         ncu="moe_p1_kernel"),
         # down (+ the split-K reduction when it runs): w2, the intermediate read once, the weighted
-        # partial row of every route written once (fp32)
-        "down": dict(bytes=touched * sh.K * sh.I * b + Rv * sh.I * bx + Rv * sh.K * 4.0,
+        # partial row of every route written once (fp32 on the bf16 path, bf16 on the mxfp8 path)
+        "down": dict(bytes=touched * sh.K * sh.I * b + Rv * sh.I * bx + Rv * sh.K * by,
                      flops=1.0 * Rv * sh.K * sh.N, name="moe_p2_kernel (down GEMM + routing weight)",
                      ncu="moe_p2_kernel"),
         # top-k reduction: every partial row read, out written, one flag per route
-        "reduce": dict(bytes=R * sh.K * 4.0 + 2.0 * sh.T * sh.K + 4.0 * R, flops=0.0,
+        "reduce": dict(bytes=R * sh.K * by + 2.0 * sh.T * sh.K + 4.0 * R, flops=0.0,
                        name="moe_combine_kernel (top-k weighted reduction)", ncu="moe_combine_kernel"),
     }
     # the whole path's algorithmic HBM bytes: touched weights, x (+ its scales) read once, out written

@@ -33,7 +33,9 @@
 //            the block's intermediate rows (TMA, one 128-row box for blocks of
 //            at least 64 rows), B = 256 rows of w2[e] (TMA, one box),
 //            D in TMEM; each epilogue thread scales its row by the routing
-//            weight and writes one fp32 row segment per route.
+//            weight and writes one row segment per route (fp32 on the bf16
+//            path; bf16 on the mxfp8 path, whose tolerance leaves room for
+//            the extra rounding).
 //   combine  out[t] = bf16(sum over the token's routes, in route order), a
 //            deterministic HBM-bound pass.
 // The weight tiles are streamed once per unit through a multi-stage shared
@@ -145,7 +147,7 @@ struct P2Params {
   const int32_t* expert_ids;
   const int32_t* ntpp;
   const float* topk_w;
-  void* yw;                 // (R, K) weighted down-projection rows, fp32
+  void* yw;                 // weighted down-projection rows, one per (route, split): fp32 (bf16 path) or bf16 (mxfp8 path)
   int32_t* flags;
   int* status;
   int K, I, E, top_k, bm, R;
@@ -964,17 +966,24 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       const uint32_t tacc = tbase + (static_cast<uint32_t>(32 * q) << 16) + static_cast<uint32_t>(buf) * 256u;
       bool released = false;
       if (32 * q < bi.nend && kFp8) {
-        // One TMEM accumulator on this path: the thread's weighted half-row
-        // (up to 4 slices of 32 fp32 features) is read into registers and the
+        // One TMEM accumulator on this path: the thread's weighted half-row is
+        // packed to bf16 in registers (up to 4 slices of 32 features) and the
         // accumulator handed back to the MMA warp before the slices go through
         // the staging buffer to global memory, as below.
         const int half = nn / 2;
         const int64_t col_base = static_cast<int64_t>(ht) * TH + h * half;
-        uint32_t yv[4][32];
+        uint32_t pk[4][16];
 #pragma unroll
-        for (int sl = 0; sl < 4; ++sl)
-          if (32 * sl < half) tmem_ld32(tacc + h * half + 32 * sl, yv[sl]);  // uniform
-        tmem_ld_wait();
+        for (int sl = 0; sl < 4; ++sl) {
+          if (32 * sl < half) {  // uniform
+            uint32_t yr[32];
+            tmem_ld32(tacc + h * half + 32 * sl, yr);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[sl][i] = pack_bf16x2(wgt * __uint_as_float(yr[2 * i]), wgt * __uint_as_float(yr[2 * i + 1]));
+          }
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -982,29 +991,21 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl) {
           if (32 * sl < half) {
+            __syncwarp();
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              __syncwarp();
+            for (int i = 0; i < 4; ++i)
+              stg4[lane * 4 + (i ^ ((lane >> 1) & 3))] =
+                  make_uint4(pk[sl][4 * i], pk[sl][4 * i + 1], pk[sl][4 * i + 2], pk[sl][4 * i + 3]);
+            __syncwarp();
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int k = 16 * hh + 4 * i;
-                stg4[lane * 4 + (i ^ ((lane >> 1) & 3))] =
-                    make_uint4(__float_as_uint(wgt * __uint_as_float(yv[sl][k])),
-                               __float_as_uint(wgt * __uint_as_float(yv[sl][k + 1])),
-                               __float_as_uint(wgt * __uint_as_float(yv[sl][k + 2])),
-                               __float_as_uint(wgt * __uint_as_float(yv[sl][k + 3])));
-              }
-              __syncwarp();
-#pragma unroll
-              for (int it = 0; it < 4; ++it) {
-                const int rl = 8 * it + (lane >> 2), cq = lane & 3;
-                const uint4 v = stg4[rl * 4 + (cq ^ ((rl >> 1) & 3))];
-                const int route_l = __shfl_sync(0xffffffffu, prow, rl);
-                const int mine_l = __shfl_sync(0xffffffffu, static_cast<int>(mine), rl);
-                if (mine_l) {
-                  const int64_t e0 = static_cast<int64_t>(route_l) * p.K + col_base + 32 * sl + 16 * hh;
-                  *reinterpret_cast<uint4*>(reinterpret_cast<float*>(p.yw) + e0 + 4 * cq) = v;
-                }
+            for (int it = 0; it < 4; ++it) {
+              const int rl = 8 * it + (lane >> 2), cq = lane & 3;
+              const uint4 v = stg4[rl * 4 + (cq ^ ((rl >> 1) & 3))];
+              const int route_l = __shfl_sync(0xffffffffu, prow, rl);
+              const int mine_l = __shfl_sync(0xffffffffu, static_cast<int>(mine), rl);
+              if (mine_l) {
+                const int64_t e0 = static_cast<int64_t>(route_l) * p.K + col_base + 32 * sl;
+                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.yw) + e0 + 8 * cq) = v;
               }
             }
           }
@@ -1075,16 +1076,49 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 // combine: out[t] = bf16( sum over j, s of yw[(t*top_k + j)*nsplit2 + s] ),
 // routes in order
 // ========================================================================
-// One thread sums 8 consecutive features of one token over its top_k routes.
-// The route flags and every route's 8 partials are loaded before any of them
-// is used (the loads of a route whose flag is 0 read workspace bytes that are
-// then discarded), so a thread has all its loads in flight at once; the sum
-// runs in route order, so the result does not depend on scheduling.
-template <int kMaxK>
-__global__ void __launch_bounds__(256, 2) moe_combine_kernel(const float* __restrict__ yw,
-                                                             const int32_t* __restrict__ flags,
-                                                             __nv_bfloat16* __restrict__ out, int T, int K,
-                                                             int top_k, int nsplit2) {
+// 8 consecutive partials of one row, kept packed in registers until they are
+// summed (bf16: one 16-byte load, fp32: two).
+template <typename TP>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 a;
+};
+template <>
+struct Raw8<float> {
+  uint4 a, b;
+};
+__device__ __forceinline__ void load_raw8(const __nv_bfloat16* p, Raw8<__nv_bfloat16>& r) {
+  r.a = __ldg(reinterpret_cast<const uint4*>(p));
+}
+__device__ __forceinline__ void load_raw8(const float* p, Raw8<float>& r) {
+  r.a = __ldg(reinterpret_cast<const uint4*>(p));
+  r.b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+}
+__device__ __forceinline__ void add_raw8(const Raw8<__nv_bfloat16>& r, float (&acc)[8]) {
+  const uint32_t w[4] = {r.a.x, r.a.y, r.a.z, r.a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] += __uint_as_float(w[i] << 16);
+    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void add_raw8(const Raw8<float>& r, float (&acc)[8]) {
+  const uint32_t w[8] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] += __uint_as_float(w[i]);
+}
+
+// One thread sums 8 consecutive features of one token over its top_k routes
+// (and their splits).  The route flags and every route's 8 partials are loaded
+// before any of them is used (the loads of a route whose flag is 0 read
+// workspace bytes that are then discarded), so a thread has all its loads in
+// flight at once; the sum runs in route order, so the result does not depend
+// on scheduling.
+template <typename TP, int kMaxK>
+__global__ void __launch_bounds__(256, sizeof(TP) == 2 ? 4 : 2)
+    moe_combine_kernel(const TP* __restrict__ yw, const int32_t* __restrict__ flags, __nv_bfloat16* __restrict__ out,
+                       int T, int K, int top_k, int nsplit2) {
   pdl_wait();  // the down phase's partial rows are read below
   const int kv = K / 8;
   const int64_t n = static_cast<int64_t>(T) * kv;
@@ -1098,26 +1132,18 @@ __global__ void __launch_bounds__(256, 2) moe_combine_kernel(const float* __rest
     const int nrows = top_k * nsplit2;
     for (int j0 = 0; j0 < nrows; j0 += kMaxK) {
       int f[kMaxK];
-      uint4 y[kMaxK][2];
+      Raw8<TP> y[kMaxK];
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j) {
         f[j] = 0;
         if (j0 + j < nrows) {
-          const int64_t r = t * nrows + j0 + j;
           f[j] = __ldg(flags + t * top_k + (j0 + j) / nsplit2);
-          const uint4* src = reinterpret_cast<const uint4*>(yw + r * K + h);
-          y[j][0] = __ldg(src);
-          y[j][1] = __ldg(src + 1);
+          load_raw8(yw + (t * nrows + j0 + j) * K + h, y[j]);
         }
       }
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j)
-        if (f[j]) {
-          const uint32_t w[8] = {y[j][0].x, y[j][0].y, y[j][0].z, y[j][0].w,
-                                 y[j][1].x, y[j][1].y, y[j][1].z, y[j][1].w};
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] += __uint_as_float(w[i]);
-        }
+        if (f[j]) add_raw8(y[j], acc);
     }
     __nv_bfloat162 o[4];
 #pragma unroll
@@ -1163,7 +1189,7 @@ static WsLayout ws_layout(bool fp8, int T, int K, int N, int E, int top_k, int b
   w.act_sf = off;
   if (fp8) off = round_up(off + (w.cap_rows / bm) * (I / 128) * kSfTileBytes, 1024);
   w.yw = off;
-  off = round_up(off + R * down_splits(fp8, T, K, N, E, top_k, bm) * K * 4, 1024);
+  off = round_up(off + R * down_splits(fp8, T, K, N, E, top_k, bm) * K * (fp8 ? 2 : 4), 1024);
   w.flags = off;
   off = round_up(off + R * 4, 1024);
   w.part = off;
@@ -1488,23 +1514,27 @@ static int run_fused(const FusedArgs& a) {
   if (err != cudaSuccess) return cuda_fail("fused_moe: down phase launch", err);
   if ((rc = mark(2)) != MOE_OK) return rc;
   // one full wave of resident blocks (grid-stride beyond it)
-  static std::atomic<int> comb_occ;  // races store the same value
-  int occ = comb_occ.load(std::memory_order_relaxed);
+  static std::atomic<int> comb_occ[2];  // races store the same value
+  int occ = comb_occ[a.fp8 ? 1 : 0].load(std::memory_order_relaxed);
   if (occ == 0) {
     int nb = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<8>, 256, 0);
+    err = a.fp8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<__nv_bfloat16, 8>, 256, 0)
+                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<float, 8>, 256, 0);
     if (err != cudaSuccess) return cuda_fail("fused_moe: combine occupancy query", err);
     occ = nb < 1 ? 1 : nb;
-    comb_occ.store(occ, std::memory_order_relaxed);
+    comb_occ[a.fp8 ? 1 : 0].store(occ, std::memory_order_relaxed);
   }
   const int64_t nvec = static_cast<int64_t>(a.T) * (a.K / 8);
   const int64_t cblocks = (nvec + 255) / 256;
   const int64_t wave = static_cast<int64_t>(occ) * nsm;
   const int cgrid = static_cast<int>(cblocks < wave ? cblocks : wave);
   cudaLaunchConfig_t c3 = config(cgrid, 256, 0);
-  err = cudaLaunchKernelEx(&c3, moe_combine_kernel<8>, reinterpret_cast<const float*>(ws + L.yw),
-                           static_cast<const int32_t*>(p1.flags), static_cast<__nv_bfloat16*>(a.out), a.T, a.K,
-                           a.top_k, p2.nsplit2);
+  __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(a.out);
+  err = a.fp8 ? cudaLaunchKernelEx(&c3, moe_combine_kernel<__nv_bfloat16, 8>,
+                                   reinterpret_cast<const __nv_bfloat16*>(ws + L.yw),
+                                   static_cast<const int32_t*>(p1.flags), outp, a.T, a.K, a.top_k, p2.nsplit2)
+              : cudaLaunchKernelEx(&c3, moe_combine_kernel<float, 8>, reinterpret_cast<const float*>(ws + L.yw),
+                                   static_cast<const int32_t*>(p1.flags), outp, a.T, a.K, a.top_k, p2.nsplit2);
   if (err != cudaSuccess) return cuda_fail("fused_moe: combine launch", err);
   return mark(3);
 }
