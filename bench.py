@@ -72,6 +72,7 @@ def parse_args(argv=None):
                     help="threads of the CPU oracle (baseline and reference arm); 0 = every host core")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay figure")
     ap.add_argument("--router", action="store_true",
                     help="start each step from router logits (moe_route_align) instead of routed ids")
     ap.add_argument("--shared", type=int, default=0,
@@ -482,8 +483,43 @@ class Problem:
         self.fused(self.plain if tune is None else tune)
 
 
+def graph_step_ms(prob: Problem, steps: int, flush=None):
+    """Device time of one step replayed from a CUDA graph (the same library launches captured once),
+    i.e. without the host's per-step submission through the Python binding; the L2 flush, when given,
+    runs between replays outside the timed windows.  None if the capture is not possible here."""
+    import torch
+
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.stream(stream):
+            prob.step()  # the first call on this stream outside the capture
+            with torch.cuda.graph(g, stream=stream):
+                prob.step()
+    except Exception:
+        torch.cuda.synchronize()
+        return None
+    torch.cuda.current_stream().wait_stream(stream)
+    cur = torch.cuda.current_stream()
+    times = []
+    for _ in range(3):
+        g.replay()
+    for _ in range(steps):
+        if flush:
+            flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(cur)
+        g.replay()
+        e1.record(cur)
+        times.append((e0, e1))
+    torch.cuda.synchronize()
+    prob.moe.moe_device_status()
+    return float(np.median([a.elapsed_time(b) for a, b in times]))
+
+
 def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barrier=None, sample_clocks=True,
-            local: int = 0):
+            local: int = 0, graph: bool = False):
     """Device time of `steps` steps after `warmup`.
 
     Pass 1 (the reported time): the steps run with nothing between their
@@ -496,7 +532,9 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
     events recorded between its launches (events between launches can keep the
     launches from overlapping, so pass 2 is used for the per-kernel times only).
     With flush_l2, pass 3 runs the steps back to back without the flush (warm
-    L2), reported beside the cold time and labelled as such.
+    L2), reported beside the cold time and labelled as such.  With graph, the
+    step is also captured once in a CUDA graph and replayed (median per step,
+    same flush policy): the device-side time without per-step host submission.
     """
     import torch
 
@@ -562,7 +600,9 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
         prob.step()  # the last flush left L2 cold; one untimed step warms it
         warm_ms = timed(cold=False) / steps
         moe.moe_device_status()
+    graph_ms = graph_step_ms(prob, steps, flush if flush_l2 else None) if graph else None
     return {"total_ms": total_ms, "ms_step": total_ms / steps, "warm_ms_step": warm_ms, "median_ms_step": median_ms,
+            "graph_ms_step": graph_ms,
             "plan_ms": sum(a.elapsed_time(e[0]) for a, e in zip(pev, ev)) / steps,
             "p1_ms": sum(e[0].elapsed_time(e[1]) for e in ev) / steps,
             "p2_ms": sum(e[1].elapsed_time(e[2]) for e in ev) / steps,
@@ -669,6 +709,10 @@ def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
         "roofline": roofline_of(sh, cm, m, peaks, peak_src),
         "gpu_launches": m["launches"],
         "clocks": m["clocks"],
+        **({"graph": {"us_per_call_median": m["graph_ms_step"] * 1e3,
+                      "note": "the same step captured once in a CUDA graph and replayed: device time without the "
+                              "host's per-step submission (not the reported value)"}}
+           if m.get("graph_ms_step") else {}),
         **({"warm": {"us_per_call": m["warm_ms_step"] * 1e3,
                      "l2": "not flushed: steps back to back, so weights can stay L2-resident (not the reported value)"}}
            if m.get("warm_ms_step") else {}),
@@ -721,7 +765,8 @@ def bench_point(sh: W.Shape, sh_w: W.Shape, inp: dict, weights: dict, args, worl
     cm = cost_model(sh_w, inp["topk_ids"], peaks)
     prob = Problem(sh, inp, dev, args.stages, args.ctas, router=args.router, n_shared=args.shared, weights=weights)
     flush = args.flush_l2 or cm["bytes_w"] < 4 * 126e6
-    m = measure(prob, args.steps, args.warmup, flush_l2=flush, barrier=barrier, local=local)
+    m = measure(prob, args.steps, args.warmup, flush_l2=flush, barrier=barrier, local=local,
+                graph=world == 1 and not args.no_graph)
     m["ms_step"] = max_over_ranks(m["ms_step"], world, dist, dev)
     line = result_line(sh, cm, m, world, args.steps, args.warmup, peaks, peak_src, flush)
     if args.router:
