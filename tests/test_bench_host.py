@@ -69,3 +69,37 @@ def test_full_algorithmic_bytes():
             + 4 * ((cap + sh.block_m - 1) // sh.block_m) + 4)
     assert cm["bytes_full"] == pytest.approx(want)
     assert cm["bytes_full"] > cm["bytes_w"]
+
+
+def test_roofline_follows_the_dominant_kernel():
+    sh = W.shape("C5", 64)
+    ids = np.tile(np.arange(sh.top_k, dtype=np.int32), (sh.T, 1))
+    peaks = dict(PEAKS, mxfp8_tflops=2928.7)
+    cm = bench.cost_model(sh, ids, peaks)
+    m = {"p1_ms": 0.01, "p2_ms": 0.05, "cb_ms": 0.002, "plan_ms": 0.003}
+    r = bench.roofline_of(sh, cm, m, peaks, "measured")
+    assert r["phase"] == "down" and r["bound"] == "hbm"
+    assert r["achieved"] == pytest.approx(cm["kernels"]["down"]["bytes"] / 0.05e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["hbm_gbs"])
+    m = {"p1_ms": 0.08, "p2_ms": 0.05, "cb_ms": 0.002, "plan_ms": 0.003}
+    assert bench.roofline_of(sh, cm, m, peaks, "measured")["phase"] == "gate_up"
+
+
+def test_mxfp8_peak_comes_from_the_committed_measurement():
+    peaks, _ = bench.load_peaks()
+    assert peaks["mxfp8_tflops"] > peaks["bf16_tflops"]
+    assert "profiles/tensor_peak_mxfp8.md" in peaks["mxfp8_source"]
+    assert bench.tensor_peak(W.shape("C3", 64), peaks) == peaks["mxfp8_tflops"]
+    assert bench.tensor_peak(W.shape("C3F4", 64), peaks) == peaks["mxfp8_tflops"]
+    assert bench.tensor_peak(W.shape("C2", 64), peaks) == peaks["bf16_tflops"]
+
+
+def test_sweep_and_headline_options():
+    a = bench.parse_args([])
+    assert a.workload == "C4" and a.tokens == 8192 and not a.sweep
+    assert bench.parse_args(["--sweep", "--sweep-workloads", "C1,C5"]).sweep
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--sweep", "--gpus", "2"])
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--sweep", "--sweep-workloads", "C9"])
+    assert bench.parse_args(["--no-graph"]).no_graph
