@@ -133,6 +133,12 @@ def tensor_peak(sh: W.Shape, peaks: dict) -> float:
     return peaks["bf16_tflops"] if sh.dtype == "bf16" else peaks.get("mxfp8_tflops", 2.0 * peaks["bf16_tflops"])
 
 
+def small_batch_default(sh: W.Shape) -> bool:
+    """Whether fused_moe_bf16 takes its small-batch form for this shape by default (the library's
+    switch: bf16, T * top_k <= 128, K and N/2 multiples of 256)."""
+    return sh.dtype == "bf16" and sh.T * sh.top_k <= 128 and sh.K % 256 == 0 and (sh.N // 2) % 256 == 0
+
+
 def cost_model(sh: W.Shape, topk_ids: np.ndarray, peaks: dict):
     """Routed FLOPs, touched weight bytes, the path roofline time (s) and each kernel's
     algorithmic bytes and FLOPs."""
@@ -166,6 +172,10 @@ def cost_model(sh: W.Shape, topk_ids: np.ndarray, peaks: dict):
         "reduce": dict(bytes=R * sh.K * by + 2.0 * sh.T * sh.K + 4.0 * R, flops=0.0,
                        name="moe_combine_kernel (top-k weighted reduction)", ncu="moe_combine_kernel"),
     }
+    if small_batch_default(sh):
+        # the small-batch form: the same bytes and FLOPs in two warp-MMA kernels, then the same combine
+        kern["gate_up"].update(name="moe_sb_up_kernel (gate/up + SwiGLU, warp MMA)", ncu="moe_sb_up_kernel")
+        kern["down"].update(name="moe_sb_down_kernel (down + routing weight, warp MMA)", ncu="moe_sb_down_kernel")
     # the whole path's algorithmic HBM bytes: touched weights, x (+ its scales) read once, out written
     # once, the routing read, the planner's arrays written (sorted ids, expert ids, the padded total)
     cap = R + sh.E * (sh.block_m - 1)
@@ -460,7 +470,9 @@ class Problem:
         self.stages, self.ctas = stages, ctas
         # planner, gate/up phase, split-K reduction, down phase, combine (+ the router kernel for
         # batches of more than 32 tokens on the router path)
-        self.launches_per_step = 5 + (1 if router and sh.T > 32 else 0)
+        # planner (+ router kernel beyond 32 tokens), then the four tensor-core launches or, for bf16
+        # with few routed rows, the two small-batch kernels and the combine (the library's default switch)
+        self.launches_per_step = (4 if small_batch_default(sh) else 5) + (1 if router and sh.T > 32 else 0)
 
     def fused(self, tune):
         m = self.moe

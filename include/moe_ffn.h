@@ -178,6 +178,14 @@ typedef struct moe_tuning {
    * call's out is undefined.  A tiny limit is a way to exercise that path;
    * it has no other use. */
   long long wait_timeout_ns;
+  /* fused_moe_bf16 only: 0 lets the library choose between the tensor-core
+   * phases and the small-batch form (two kernels that stream each touched
+   * weight row once through warp-level MMAs, then the same top-k combine;
+   * taken by default when T * top_k <= 128); 1 takes the small-batch form
+   * whenever the shapes allow it (K and N/2 multiples of 256, T <= 8192);
+   * -1 never.  Both give the same result within the bf16 tolerance; the
+   * phase events then mark its gate/up kernel, down kernel and combine. */
+  int small_batch;
 } moe_tuning;
 
 /* ------------------------------------------------------------------------
@@ -195,6 +203,11 @@ typedef struct moe_tuning {
  *                 outputs for the same (T, top_k, E, block_m, capacity).
  * Constraints: K % 128 == 0, N % 16 == 0, N >= 16, block_m in {16, 32, 64,
  * 128}; every pointer 16-byte aligned, workspace 256-byte aligned.
+ * Small batches ([RFC] Background: decode-sized calls stream their experts'
+ * weights with little arithmetic per byte) -- T * top_k <= 128 with K and
+ * N/2 multiples of 256, or as moe_tuning.small_batch says -- run as two
+ * weight-streaming kernels (warp-level MMAs) after the planner, then the
+ * same combine: the same result up to fp32 summation order, deterministic.
  * ---------------------------------------------------------------------- */
 MOE_API int fused_moe_bf16(const void* x, const void* w1, const void* w2,
                    const int32_t* sorted_token_ids, const int32_t* expert_ids,

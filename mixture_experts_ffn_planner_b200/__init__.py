@@ -64,7 +64,8 @@ class MoeError(RuntimeError):
 class Tuning(ctypes.Structure):
     """``moe_tuning``: 0 in a field keeps the library's default."""
     _fields_ = [("stages", ctypes.c_int), ("num_ctas", ctypes.c_int),
-                ("phase_events", ctypes.POINTER(ctypes.c_void_p)), ("wait_timeout_ns", ctypes.c_longlong)]
+                ("phase_events", ctypes.POINTER(ctypes.c_void_p)), ("wait_timeout_ns", ctypes.c_longlong),
+                ("small_batch", ctypes.c_int)]
 
     @staticmethod
     def with_events(events, stages: int = 0, num_ctas: int = 0) -> "Tuning":

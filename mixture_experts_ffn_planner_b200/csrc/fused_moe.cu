@@ -49,6 +49,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "small_batch.h"
 
 namespace moe {
 
@@ -1341,6 +1342,45 @@ static int check_fused(const FusedArgs& a, bool has_ws) {
   return MOE_OK;
 }
 
+// The top-k reduction: one wave of resident blocks of the combine kernel
+// (grid-stride beyond it) over the partial rows `yw` (bf16 when `bf16_parts`,
+// else fp32; nsplit2 per route) and the route flags.  Chained to the
+// previous launch by programmatic dependent launch.
+static int launch_combine(bool bf16_parts, const uint8_t* yw, const int32_t* flags, void* out, int T, int K,
+                          int top_k, int nsplit2, int nsm, cudaStream_t stream) {
+  static std::atomic<int> comb_occ[2];  // races store the same value
+  int occ = comb_occ[bf16_parts ? 1 : 0].load(std::memory_order_relaxed);
+  cudaError_t err;
+  if (occ == 0) {
+    int nb = 0;
+    err = bf16_parts
+              ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<__nv_bfloat16, 8>, 256, 0)
+              : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<float, 8>, 256, 0);
+    if (err != cudaSuccess) return cuda_fail("fused_moe: combine occupancy query", err);
+    occ = nb < 1 ? 1 : nb;
+    comb_occ[bf16_parts ? 1 : 0].store(occ, std::memory_order_relaxed);
+  }
+  const int64_t nvec = static_cast<int64_t>(T) * (K / 8);
+  const int64_t cblocks = (nvec + 255) / 256;
+  const int64_t wave = static_cast<int64_t>(occ) * nsm;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t c3 = {};
+  c3.gridDim = dim3(static_cast<unsigned>(cblocks < wave ? cblocks : wave), 1, 1);
+  c3.blockDim = dim3(256, 1, 1);
+  c3.stream = stream;
+  c3.attrs = pdl;
+  c3.numAttrs = 1;
+  __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(out);
+  err = bf16_parts ? cudaLaunchKernelEx(&c3, moe_combine_kernel<__nv_bfloat16, 8>,
+                                        reinterpret_cast<const __nv_bfloat16*>(yw), flags, outp, T, K, top_k, nsplit2)
+                   : cudaLaunchKernelEx(&c3, moe_combine_kernel<float, 8>, reinterpret_cast<const float*>(yw), flags,
+                                        outp, T, K, top_k, nsplit2);
+  if (err != cudaSuccess) return cuda_fail("fused_moe: combine launch", err);
+  return MOE_OK;
+}
+
 static int run_fused(const FusedArgs& a) {
   const char* nm = a.w_fp4 ? "fused_moe_mxfp4" : (a.fp8 ? "fused_moe_mxfp8" : "fused_moe_bf16");
   int rc0 = check_fused(a, true);
@@ -1352,6 +1392,9 @@ static int run_fused(const FusedArgs& a) {
 
   const int I = a.N / 2;
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  // Blocks a kernel may visit: never past the caller's sorted_token_ids /
+  // expert_ids arrays, even if num_tokens_post_padded were out of range.
+  const int max_blocks = static_cast<int>(std::min<int64_t>(L.cap_rows, a.capacity) / a.bm);
   static std::atomic<int*> status_ptr[kMaxDevices];  // per device; races store the same address
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice");
@@ -1364,8 +1407,37 @@ static int run_fused(const FusedArgs& a) {
     status_ptr[dev].store(status, std::memory_order_relaxed);
   }
 
-  CUtensorMap tm_w1, tm_w2, tm_w2x, tm_act, tm_actx;
   int rc;
+  const unsigned long long wait_ns =
+      a.tune && a.tune->wait_timeout_ns > 0 ? static_cast<unsigned long long>(a.tune->wait_timeout_ns) : kWaitTimeoutNs;
+  const int nsm = sm_count();
+  if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(SM count)");
+  if (!a.fp8) {
+    const int mode = a.tune ? a.tune->small_batch : 0;
+    const bool small = mode >= 0 && small_batch_shapes_ok(a.T, a.K, a.N, a.top_k) &&
+                       (mode > 0 || static_cast<int64_t>(a.T) * a.top_k <= kSbAutoRoutes);
+    if (small) {
+      SbArgs sb{};
+      sb.x = a.x; sb.w1 = a.w1; sb.w2 = a.w2;
+      sb.sorted_ids = a.sorted_ids; sb.expert_ids = a.expert_ids; sb.ntpp = a.ntpp;
+      sb.topk_w = a.topk_w;
+      sb.T = a.T; sb.K = a.K; sb.N = a.N; sb.E = a.E; sb.top_k = a.top_k; sb.bm = a.bm;
+      sb.max_blocks = max_blocks;
+      sb.act = ws + L.act;
+      sb.yw = reinterpret_cast<float*>(ws + L.yw);
+      sb.flags = reinterpret_cast<int32_t*>(ws + L.flags);
+      sb.pf_all = static_cast<int64_t>(a.E) * (a.N + I) * a.K * 2 <= kPrefetchAllBytes;
+      void* const* ev = a.tune ? a.tune->phase_events : nullptr;
+      if ((rc = run_small_batch(sb, a.stream, ev)) != MOE_OK) return rc;
+      if ((rc = launch_combine(false, ws + L.yw, sb.flags, a.out, a.T, a.K, a.top_k, 1, nsm, a.stream)) != MOE_OK)
+        return rc;
+      if (ev && cudaEventRecord(static_cast<cudaEvent_t>(ev[3]), a.stream) != cudaSuccess)
+        return cuda_fail("fused_moe: cudaEventRecord");
+      return MOE_OK;
+    }
+  }
+
+  CUtensorMap tm_w1, tm_w2, tm_w2x, tm_act, tm_actx;
   const TmapKind wk = a.w_fp4 ? kTmFp4 : (a.fp8 ? kTmU8 : kTmBf16), ak = a.fp8 ? kTmU8 : kTmBf16;
   if ((rc = make_tmap(&tm_w1, a.w1, wk, static_cast<int64_t>(a.E) * a.N, a.K, 128)) != MOE_OK) return rc;
   if ((rc = make_tmap(&tm_w2, a.w2, wk, static_cast<int64_t>(a.E) * a.K, I, 128)) != MOE_OK) return rc;
@@ -1379,15 +1451,8 @@ static int run_fused(const FusedArgs& a) {
     return rc;
   if (a_rows >= kM && (rc = make_tmap(&tm_actx, ws + L.act, ak, L.cap_rows, I, 128)) != MOE_OK) return rc;
 
-  const int nsm = sm_count();
-  if (nsm <= 0) return cuda_fail("cudaDeviceGetAttribute(SM count)");
   const int req_stages = a.tune ? a.tune->stages : 0;
-  const unsigned long long wait_ns =
-      a.tune && a.tune->wait_timeout_ns > 0 ? static_cast<unsigned long long>(a.tune->wait_timeout_ns) : kWaitTimeoutNs;
   const int req_ctas = a.tune ? a.tune->num_ctas : 0;
-  // Blocks a kernel may visit: never past the caller's sorted_token_ids /
-  // expert_ids arrays, even if num_tokens_post_padded were out of range.
-  const int max_blocks = static_cast<int>(std::min<int64_t>(L.cap_rows, a.capacity) / a.bm);
 
   P1Params p1{};
   p1.x = static_cast<const uint8_t*>(a.x);
@@ -1513,29 +1578,9 @@ static int run_fused(const FusedArgs& a) {
               : cudaLaunchKernelEx(&c2, moe_p2_kernel<false>, tm_w2, tm_w2x, tm_act, tm_actx, p2);
   if (err != cudaSuccess) return cuda_fail("fused_moe: down phase launch", err);
   if ((rc = mark(2)) != MOE_OK) return rc;
-  // one full wave of resident blocks (grid-stride beyond it)
-  static std::atomic<int> comb_occ[2];  // races store the same value
-  int occ = comb_occ[a.fp8 ? 1 : 0].load(std::memory_order_relaxed);
-  if (occ == 0) {
-    int nb = 0;
-    err = a.fp8 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<__nv_bfloat16, 8>, 256, 0)
-                : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, moe_combine_kernel<float, 8>, 256, 0);
-    if (err != cudaSuccess) return cuda_fail("fused_moe: combine occupancy query", err);
-    occ = nb < 1 ? 1 : nb;
-    comb_occ[a.fp8 ? 1 : 0].store(occ, std::memory_order_relaxed);
-  }
-  const int64_t nvec = static_cast<int64_t>(a.T) * (a.K / 8);
-  const int64_t cblocks = (nvec + 255) / 256;
-  const int64_t wave = static_cast<int64_t>(occ) * nsm;
-  const int cgrid = static_cast<int>(cblocks < wave ? cblocks : wave);
-  cudaLaunchConfig_t c3 = config(cgrid, 256, 0);
-  __nv_bfloat16* outp = static_cast<__nv_bfloat16*>(a.out);
-  err = a.fp8 ? cudaLaunchKernelEx(&c3, moe_combine_kernel<__nv_bfloat16, 8>,
-                                   reinterpret_cast<const __nv_bfloat16*>(ws + L.yw),
-                                   static_cast<const int32_t*>(p1.flags), outp, a.T, a.K, a.top_k, p2.nsplit2)
-              : cudaLaunchKernelEx(&c3, moe_combine_kernel<float, 8>, reinterpret_cast<const float*>(ws + L.yw),
-                                   static_cast<const int32_t*>(p1.flags), outp, a.T, a.K, a.top_k, p2.nsplit2);
-  if (err != cudaSuccess) return cuda_fail("fused_moe: combine launch", err);
+  if ((rc = launch_combine(a.fp8, ws + L.yw, static_cast<const int32_t*>(p1.flags), a.out, a.T, a.K, a.top_k,
+                           p2.nsplit2, nsm, a.stream)) != MOE_OK)
+    return rc;
   return mark(3);
 }
 
