@@ -78,6 +78,9 @@ def parse_args(argv=None):
     ap.add_argument("--shared", type=int, default=0,
                     help="shared experts after the routed ones (every token, weight 1); needs --router")
     ap.add_argument("--stages", type=int, default=0)
+    ap.add_argument("--small-batch", choices=["auto", "on", "off"], default="auto",
+                    help="bf16: the library's choice between the small-batch form and the tensor-core phases "
+                         "(moe_tuning.small_batch)")
     ap.add_argument("--ctas", type=int, default=0)
     ap.add_argument("--flush-l2", action="store_true",
                     help="flush L2 between steps (automatic when the touched weights are < 4x L2)")
@@ -133,13 +136,17 @@ def tensor_peak(sh: W.Shape, peaks: dict) -> float:
     return peaks["bf16_tflops"] if sh.dtype == "bf16" else peaks.get("mxfp8_tflops", 2.0 * peaks["bf16_tflops"])
 
 
-def small_batch_default(sh: W.Shape) -> bool:
-    """Whether fused_moe_bf16 takes its small-batch form for this shape by default (the library's
-    switch: bf16, T * top_k <= 128, K and N/2 multiples of 256)."""
-    return sh.dtype == "bf16" and sh.T * sh.top_k <= 128 and sh.K % 256 == 0 and (sh.N // 2) % 256 == 0
+SMALL_BATCH_MODE = {"auto": 0, "on": 1, "off": -1}
 
 
-def cost_model(sh: W.Shape, topk_ids: np.ndarray, peaks: dict):
+def small_batch_form(sh: W.Shape, mode: int = 0) -> bool:
+    """Whether fused_moe_bf16 takes its small-batch form for this shape under moe_tuning.small_batch =
+    mode (the library's switch: bf16, K and N/2 multiples of 256, and by default T * top_k <= 128)."""
+    ok = sh.dtype == "bf16" and sh.K % 256 == 0 and (sh.N // 2) % 256 == 0 and sh.T <= 8192
+    return ok and mode >= 0 and (mode > 0 or sh.T * sh.top_k <= 128)
+
+
+def cost_model(sh: W.Shape, topk_ids: np.ndarray, peaks: dict, small_batch: int = 0):
     """Routed FLOPs, touched weight bytes, the path roofline time (s) and each kernel's
     algorithmic bytes and FLOPs."""
     R = sh.T * sh.top_k
@@ -172,7 +179,7 @@ def cost_model(sh: W.Shape, topk_ids: np.ndarray, peaks: dict):
         "reduce": dict(bytes=R * sh.K * by + 2.0 * sh.T * sh.K + 4.0 * R, flops=0.0,
                        name="moe_combine_kernel (top-k weighted reduction)", ncu="moe_combine_kernel"),
     }
-    if small_batch_default(sh):
+    if small_batch_form(sh, small_batch):
         # the small-batch form: the same bytes and FLOPs in two warp-MMA kernels, then the same combine
         kern["gate_up"].update(name="moe_sb_up_kernel (gate/up + SwiGLU, warp MMA)", ncu="moe_sb_up_kernel")
         kern["down"].update(name="moe_sb_down_kernel (down + routing weight, warp MMA)", ncu="moe_sb_down_kernel")
@@ -427,7 +434,7 @@ class Problem:
     """Device-resident inputs of one workload and one step of the hot path."""
 
     def __init__(self, sh: W.Shape, inp: dict, dev, stages: int = 0, ctas: int = 0, router: bool = False,
-                 n_shared: int = 0, weights: dict | None = None):
+                 n_shared: int = 0, weights: dict | None = None, small_batch: int = 0):
         import torch
 
         import mixture_experts_ffn_planner_b200 as moe
@@ -467,12 +474,13 @@ class Problem:
         self.ws = torch.empty(moe.moe_workspace_bytes(dt, sh.T, sh.K, sh.N, sh.E + n_shared, sh.top_k + n_shared, bm),
                               dtype=torch.uint8, device=dev)
         self.plain = moe.Tuning(stages, ctas, None)
-        self.stages, self.ctas = stages, ctas
+        self.plain.small_batch = small_batch
+        self.stages, self.ctas, self.small_batch = stages, ctas, small_batch
         # planner, gate/up phase, split-K reduction, down phase, combine (+ the router kernel for
         # batches of more than 32 tokens on the router path)
         # planner (+ router kernel beyond 32 tokens), then the four tensor-core launches or, for bf16
         # with few routed rows, the two small-batch kernels and the combine (the library's default switch)
-        self.launches_per_step = (4 if small_batch_default(sh) else 5) + (1 if router and sh.T > 32 else 0)
+        self.launches_per_step = (4 if small_batch_form(sh, small_batch) else 5) + (1 if router and sh.T > 32 else 0)
 
     def fused(self, tune):
         m = self.moe
@@ -605,6 +613,8 @@ def measure(prob: Problem, steps: int, warmup: int, flush_l2: bool = False, barr
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     pev = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     tunes = [moe.Tuning.with_events(e, prob.stages, prob.ctas) for e in ev]
+    for t in tunes:
+        t.small_batch = prob.small_batch
     timed(tunes, pev)
     moe.moe_device_status()
     warm_ms = None
@@ -693,7 +703,7 @@ def roofline_of(sh: W.Shape, cm: dict, m: dict, peaks: dict, peak_src: str):
             "peak_source": src, "algorithmic_flops_per_launch": k["flops"]}
 
 
-def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
+def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2, small_batch: int = 0):
     ms_step = m["ms_step"]
     l2 = ("L2 flushed between steps (512 MB written then read back, outside the per-step events)" if flush_l2 else
           f"inputs larger than L2 (touched expert weights {cm['bytes_w'] / 1e9:.2f} GB per step)")
@@ -704,7 +714,8 @@ def result_line(sh, cm, m, world, steps, warmup, peaks, peak_src, flush_l2):
         "data": "synthetic (seeded workloads generator, random weights)",
         "config": {"workload": f"{sh.name}: {sh.dtype} MoE FFN K={sh.K} N={sh.N} (intermediate {sh.I}) "
                                f"E={sh.E} top_k={sh.top_k} T={sh.T} block_m={sh.block_m}",
-                   "tokens_per_gpu": sh.T, "parallelism": f"replicas x{world}", "l2": l2},
+                   "tokens_per_gpu": sh.T, "parallelism": f"replicas x{world}", "l2": l2,
+                   "form": "small-batch (warp MMA)" if small_batch_form(sh, small_batch) else "tcgen05 phases"},
         "us_per_call": ms_step * 1e3,
         **({"us_per_call_median": m["median_ms_step"] * 1e3} if m.get("median_ms_step") else {}),
         "weight_GBps": cm["bytes_w"] / (ms_step * 1e-3) / 1e9,
@@ -774,13 +785,15 @@ def _setup_inputs(sh: W.Shape, args, rank: int, world: int, dist, dev, need_host
 def bench_point(sh: W.Shape, sh_w: W.Shape, inp: dict, weights: dict, args, world: int, rank: int, local: int,
                 dist, dev, peaks, peak_src, barrier, cpu_seconds: float):
     """Measures one workload and returns its JSON line (rank 0 prints it)."""
-    cm = cost_model(sh_w, inp["topk_ids"], peaks)
-    prob = Problem(sh, inp, dev, args.stages, args.ctas, router=args.router, n_shared=args.shared, weights=weights)
+    cm = cost_model(sh_w, inp["topk_ids"], peaks, SMALL_BATCH_MODE[args.small_batch])
+    prob = Problem(sh, inp, dev, args.stages, args.ctas, router=args.router, n_shared=args.shared, weights=weights,
+                   small_batch=SMALL_BATCH_MODE[args.small_batch])
     flush = args.flush_l2 or cm["bytes_w"] < 4 * 126e6
     m = measure(prob, args.steps, args.warmup, flush_l2=flush, barrier=barrier, local=local,
                 graph=world == 1 and not args.no_graph)
     m["ms_step"] = max_over_ranks(m["ms_step"], world, dist, dev)
-    line = result_line(sh, cm, m, world, args.steps, args.warmup, peaks, peak_src, flush)
+    line = result_line(sh, cm, m, world, args.steps, args.warmup, peaks, peak_src, flush,
+                       SMALL_BATCH_MODE[args.small_batch])
     if args.router:
         line["config"]["router"] = "in the step: moe_route_align (softmax, top-k, renormalise) from fp32 logits"
     if args.shared:

@@ -18,10 +18,11 @@
 //     added in warp order, and bf16(silu(gate) * up) goes to the
 //     intermediate -- the same values, in the same layout, as the gate/up
 //     phase of the tensor path.  It also clears the route flags.
-//   moe_sb_down_kernel: one warp per (planner block, 16 output features):
-//     those 16 rows of w2[e] against the block's intermediate rows; each
-//     routed row's 16 weighted fp32 sums go to its partial row and its
-//     route flag is set.
+//   moe_sb_down_kernel: one item per (planner block, 16 output features):
+//     those 16 rows of w2[e] against the block's intermediate rows -- a CTA
+//     per item with the N/2 reduction split over its 8 warps the same way
+//     when N/2 >= 512, else a warp per item; each routed row's 16 weighted
+//     fp32 sums go to its partial row and its route flag is set.
 //   The combine kernel then sums each token's partial rows in route order
 //   (fp32, one bf16 rounding), exactly as after the tensor-core phases.
 //
@@ -257,10 +258,102 @@ __global__ void __launch_bounds__(kSbThreads, 2) moe_sb_up_kernel(const __grid_c
 }
 
 // Down projection of 16 output features k0 .. k0+15 for up to 8 * NT routed
+// rows of the block: every warp of the CTA takes N/16 of the N/2-long
+// reduction, the partial tiles are added in warp order by warp 0, whose
+// thread (g, q) ends with features k0 + g and k0 + g + 8 of rows 2q, 2q + 1
+// of every tile, weighted into the rows' partial rows.
+template <int NT>
+__device__ __forceinline__ void sb_down_tile(const SbParams& p, int e, int k0, const int* row, const int* route,
+                                             int ng, int warp, int lane, float (*red)[2][32][4]) {
+  const int g = lane >> 2, q = lane & 3;
+  const int iw = p.I / kSbWarps;  // a multiple of 32
+  const __nv_bfloat16* ra = p.w2 + (static_cast<int64_t>(e) * p.K + k0 + g) * p.I + warp * iw;
+  const __nv_bfloat16* rb = ra + static_cast<int64_t>(8) * p.I;
+  const __nv_bfloat16* bn[NT];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int i = 8 * t + g;
+    bn[t] = p.act + static_cast<int64_t>(row[i < ng ? i : ng - 1]) * p.I + warp * iw;
+  }
+  float d[NT][4];
+  sb_mma_rows<NT, true>(ra, rb, bn, iw, q, d);
+#pragma unroll
+  for (int t = 0; t < NT; ++t)
+    *reinterpret_cast<float4*>(red[warp][t][lane]) = make_float4(d[t][0], d[t][1], d[t][2], d[t][3]);
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int w = 0; w < kSbWarps; ++w) {
+        const float4 v = *reinterpret_cast<const float4*>(red[w][t][lane]);
+        s4[0] += v.x;
+        s4[1] += v.y;
+        s4[2] += v.z;
+        s4[3] += v.w;
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int i = 8 * t + 2 * q + h;
+        if (i < ng) {
+          const int rt = route[i];
+          const float w = __ldg(p.topk_w + rt);
+          float* y = p.yw + static_cast<int64_t>(rt) * p.K + k0 + g;
+          y[0] = w * s4[h];
+          y[8] = w * s4[2 + h];
+        }
+      }
+    }
+  }
+  __syncthreads();  // red is reused by the next tile
+}
+
+__device__ __forceinline__ void sb_down_per_cta(const SbParams& p) {
+  __shared__ int s_tok[kSbMaxBm], s_row[kSbMaxBm], s_route[kSbMaxBm];
+  __shared__ __align__(16) float s_red[kSbWarps][2][32][4];
+  __shared__ int s_nr, s_e;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // contiguous ranges of (block, 16-feature group) items per CTA
+  const int n_fg = p.K / 16;
+  const int64_t n_items = static_cast<int64_t>(sb_num_blocks(p)) * n_fg;
+  const int64_t per = (n_items + gridDim.x - 1) / gridDim.x;
+  const int64_t it0 = per * blockIdx.x, it1 = it0 + per < n_items ? it0 + per : n_items;
+  int cur_b = -1;
+  for (int64_t it = it0; it < it1; ++it) {
+    const int b = static_cast<int>(it / n_fg);
+    const int k0 = 16 * static_cast<int>(it - static_cast<int64_t>(b) * n_fg);
+    if (b != cur_b) {  // the same in every warp
+      cur_b = b;
+      __syncthreads();  // every warp has read the previous block's row count and rows
+      if (warp == 0) {
+        const int e = __ldg(p.expert_ids + b);
+        const int n = sb_block_rows(p, b, e, s_tok, s_row, s_route, lane);
+        if (lane == 0) {
+          s_nr = n;
+          s_e = e;
+        }
+      }
+      __syncthreads();
+    }
+    const int nr = s_nr, e = s_e;
+    for (int r0 = 0; r0 < nr; r0 += 16) {
+      const int ng = nr - r0 < 16 ? nr - r0 : 16;
+      if (ng <= 8)
+        sb_down_tile<1>(p, e, k0, s_row + r0, s_route + r0, ng, warp, lane, s_red);
+      else
+        sb_down_tile<2>(p, e, k0, s_row + r0, s_route + r0, ng, warp, lane, s_red);
+    }
+    if (k0 == 0 && warp == 0)
+      for (int i = lane; i < nr; i += 32) p.flags[s_route[i]] = 1;
+  }
+}
+
+// Warp-per-item schedule of the down projection (below).
+// Down projection of 16 output features k0 .. k0+15 for up to 8 * NT routed
 // rows of the block: thread (g, q) ends with features k0 + g and k0 + g + 8
 // of rows 2q, 2q + 1 of every tile, weighted into the rows' partial rows.
 template <int NT>
-__device__ __forceinline__ void sb_down_tile(const SbParams& p, int e, int k0, const int* row, const int* route,
+__device__ __forceinline__ void sb_down_tile_warp(const SbParams& p, int e, int k0, const int* row, const int* route,
                                              int ng, int lane) {
   const int g = lane >> 2, q = lane & 3;
   const __nv_bfloat16* ra = p.w2 + (static_cast<int64_t>(e) * p.K + k0 + g) * p.I;
@@ -288,11 +381,9 @@ __device__ __forceinline__ void sb_down_tile(const SbParams& p, int e, int k0, c
     }
 }
 
-__global__ void __launch_bounds__(kSbThreads, 2) moe_sb_down_kernel(const __grid_constant__ SbParams p) {
+__device__ __forceinline__ void sb_down_per_warp(const SbParams& p) {
   __shared__ int s_tok[kSbWarps][kSbMaxBm], s_row[kSbWarps][kSbMaxBm], s_route[kSbWarps][kSbMaxBm];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_wait();  // the intermediate and the cleared flags are read below
-  pdl_launch_dependents();
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nw = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5, gw = gtid >> 5;
   const int n_fg = p.K / 16;  // groups of 16 output features
@@ -311,19 +402,34 @@ __global__ void __launch_bounds__(kSbThreads, 2) moe_sb_down_kernel(const __grid
     for (int r0 = 0; r0 < nr; r0 += 16) {
       const int ng = nr - r0 < 16 ? nr - r0 : 16;
       if (ng <= 8)
-        sb_down_tile<1>(p, e, k0, s_row[warp] + r0, s_route[warp] + r0, ng, lane);
+        sb_down_tile_warp<1>(p, e, k0, s_row[warp] + r0, s_route[warp] + r0, ng, lane);
       else
-        sb_down_tile<2>(p, e, k0, s_row[warp] + r0, s_route[warp] + r0, ng, lane);
+        sb_down_tile_warp<2>(p, e, k0, s_row[warp] + r0, s_route[warp] + r0, ng, lane);
     }
     if (k0 == 0)
       for (int i = lane; i < nr; i += 32) p.flags[s_route[warp][i]] = 1;
   }
 }
 
+// One kernel, two schedules: a CTA per item (the reduction split over its
+// warps) when N/2 is long enough to give every warp several 32-value blocks,
+// else a warp per item (N/2 = 256: one block per warp would leave each item
+// a chain of barriers around a single load).
+template <bool kPerCta>
+__global__ void __launch_bounds__(kSbThreads, 2) moe_sb_down_kernel(const __grid_constant__ SbParams p) {
+  pdl_wait();  // the intermediate and the cleared flags are read below
+  pdl_launch_dependents();
+  if (kPerCta)
+    sb_down_per_cta(p);
+  else
+    sb_down_per_warp(p);
+}
+
 }  // namespace
 
 bool small_batch_shapes_ok(int T, int K, int N, int top_k) {
   (void)top_k;
+  // K and N/2 split into 8 warp shares of whole 32-value blocks
   return T > 0 && T <= kSbMaxT && K % 256 == 0 && N % 2 == 0 && (N / 2) % 256 == 0;
 }
 
@@ -365,7 +471,8 @@ int run_small_batch(const SbArgs& a, cudaStream_t stream, void* const* ev) {
   cudaError_t err = cudaLaunchKernelEx(&c, moe_sb_up_kernel, p);
   if (err != cudaSuccess) return cuda_fail("fused_moe_bf16: small-batch gate/up launch", err);
   if ((rc = mark(1)) != MOE_OK) return rc;
-  err = cudaLaunchKernelEx(&c, moe_sb_down_kernel, p);
+  err = p.I >= 512 ? cudaLaunchKernelEx(&c, moe_sb_down_kernel<true>, p)
+                   : cudaLaunchKernelEx(&c, moe_sb_down_kernel<false>, p);
   if (err != cudaSuccess) return cuda_fail("fused_moe_bf16: small-batch down launch", err);
   return mark(2);
 }
