@@ -255,17 +255,19 @@ class ClockSampler:
 
 def kernel_traffic(kernel: str, workload_tag: str):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (its sha256 is recorded in the summary)."""
+    the current kernel source (the summary records the sha256 of the source
+    file, csrc/fused_moe.cu unless it names another with ``source_file:``)."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload_tag}.md")
     if not os.path.exists(path):
         return None
     txt = open(path).read()
     m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
     h = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    f = re.search(r"source_file:\s*(\S+)", txt)
     if not m or not h:
         return None
-    src = os.path.join(ROOT, "mixture_experts_ffn_planner_b200", "csrc", "fused_moe.cu")
-    if hashlib.sha256(open(src, "rb").read()).hexdigest() != h.group(1):
+    src = os.path.join(ROOT, "mixture_experts_ffn_planner_b200", "csrc", f.group(1) if f else "fused_moe.cu")
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != h.group(1):
         return None
     return float(m.group(1))
 

@@ -103,3 +103,25 @@ def test_sweep_and_headline_options():
     with pytest.raises(SystemExit):
         bench.parse_args(["--sweep", "--sweep-workloads", "C9"])
     assert bench.parse_args(["--no-graph"]).no_graph
+
+
+def test_kernel_traffic_is_dropped_when_its_source_changes(tmp_path, monkeypatch):
+    """A profile's DRAM bytes count only while the source file it names is unchanged."""
+    import hashlib
+
+    csrc = tmp_path / "mixture_experts_ffn_planner_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "small_batch.cu").write_text("kernel a")
+    (csrc / "fused_moe.cu").write_text("kernel b")
+    (tmp_path / "profiles").mkdir()
+    sha_a = hashlib.sha256(b"kernel a").hexdigest()
+    sha_b = hashlib.sha256(b"kernel b").hexdigest()
+    (tmp_path / "profiles" / "k_W.md").write_text(
+        f"dram_bytes_per_launch: 1.5e9\nsource_file: small_batch.cu\nsource_sha256: {sha_a}\n")
+    (tmp_path / "profiles" / "j_W.md").write_text(f"dram_bytes_per_launch: 2.5e9\nsource_sha256: {sha_b}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.kernel_traffic("k", "W") == 1.5e9
+    assert bench.kernel_traffic("j", "W") == 2.5e9          # no source_file: fused_moe.cu
+    (csrc / "small_batch.cu").write_text("kernel a, changed")
+    assert bench.kernel_traffic("k", "W") is None
+    assert bench.kernel_traffic("missing", "W") is None
