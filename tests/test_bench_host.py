@@ -125,3 +125,19 @@ def test_kernel_traffic_is_dropped_when_its_source_changes(tmp_path, monkeypatch
     (csrc / "small_batch.cu").write_text("kernel a, changed")
     assert bench.kernel_traffic("k", "W") is None
     assert bench.kernel_traffic("missing", "W") is None
+
+
+def test_small_batch_form_follows_the_library_switch():
+    """The bench's launch count and kernel names follow fused_moe_bf16's choice of form: bf16 with K and
+    N/2 multiples of 256, by default when T * top_k <= 128; forced on or off by moe_tuning.small_batch."""
+    c1, c5_8, c5_64, c3 = W.shape("C1", 64), W.shape("C5", 8), W.shape("C5", 64), W.shape("C3", 64)
+    assert bench.small_batch_form(c1) and bench.small_batch_form(c5_8)
+    assert not bench.small_batch_form(c5_64)                 # 512 routed rows
+    assert bench.small_batch_form(c5_64, 1) and not bench.small_batch_form(c1, -1)
+    assert not bench.small_batch_form(c3, 1)                 # mxfp8 has no small-batch form
+    odd = W.Shape(name="S", dtype="bf16", T=4, K=384, N=512, E=4, top_k=2, block_m=64)
+    assert not bench.small_batch_form(odd, 1)                # K not a multiple of 256
+    ids = np.zeros((c1.T, c1.top_k), np.int32)
+    names = bench.cost_model(c1, ids, PEAKS)["kernels"]
+    assert names["gate_up"]["ncu"] == "moe_sb_up_kernel" and names["down"]["ncu"] == "moe_sb_down_kernel"
+    assert bench.cost_model(c1, ids, PEAKS, small_batch=-1)["kernels"]["gate_up"]["ncu"] == "moe_p1_kernel"
