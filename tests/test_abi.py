@@ -156,3 +156,27 @@ def test_noalloc_rejects_like_fused_bf16(lib):
         assert _noalloc(lib, **kw) == code, kw
         assert _bf16(lib, **kw) == code, kw
     assert _noalloc(lib, T=0) == OK
+
+
+def test_tuning_struct_layout_matches_the_header(tmp_path):
+    """The binding's ctypes moe_tuning has the C struct's size and field offsets (compiled from
+    include/moe_ffn.h with the host C compiler)."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    fields = [f[0] for f in moe.Tuning._fields_]
+    prog = tmp_path / "layout.c"
+    prog.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "moe_ffn.h"\nint main(void) {\n'
+                    '  printf("size %zu\\n", sizeof(moe_tuning));\n'
+                    + "".join(f'  printf("{f} %zu\\n", offsetof(moe_tuning, {f}));\n' for f in fields)
+                    + "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(prog), "-o", str(exe)], check=True)
+    got = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                        check=True).stdout.splitlines())
+    assert int(got["size"]) == ctypes.sizeof(moe.Tuning)
+    for f in fields:
+        assert int(got[f]) == getattr(moe.Tuning, f).offset, f
